@@ -1,0 +1,147 @@
+"""NumPy front end of the CPU oracle (adamas_oracle.c) -- TEST INFRASTRUCTURE ONLY.
+
+Only the tests, the package smoke check and the bench's CPU-baseline leg may
+import this module.  The product path never does.
+
+The C source follows the ADAMAS long-context sparse attention article
+(lnwmold.com/news/826806): §2.1 Hadamard rotation, §2.2 dynamic 2-bit bucketing,
+§3.1 packing of the code cache, §2.3 Manhattan-distance scoring, §5.2 token budget,
+followed by exact attention over the kept rows.  Parity unpinned: the page's own
+activation statistics and accuracy tables (they need model weights and datasets).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+SOURCE = os.path.join(_HERE, "adamas_oracle.c")
+LIBRARY = os.path.join(_HERE, "liboracle.so")
+CFLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared", "-pthread"]
+
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile adamas_oracle.c into liboracle.so next to it (gcc, no fast-math, no FMA contraction)."""
+    if force or not os.path.exists(LIBRARY) or os.path.getmtime(LIBRARY) < os.path.getmtime(SOURCE):
+        tmp = LIBRARY + f".tmp{os.getpid()}"
+        subprocess.run(["gcc", *CFLAGS, "-o", tmp, SOURCE, "-lm"], check=True)
+        os.replace(tmp, LIBRARY)
+    return LIBRARY
+
+
+def lib():
+    global _lib
+    with _lock:
+        if _lib is None:
+            l = ctypes.CDLL(build())
+            P = ctypes.c_void_p
+            I64, I32 = ctypes.c_int64, ctypes.c_int
+            l.oracle_rotate.argtypes = [P, I64, I32, P]
+            l.oracle_bucket_pack.argtypes = [P, I64, I32, P]
+            l.oracle_encode.argtypes = [P, I64, I32, P]
+            l.oracle_distance.argtypes = [P, P, I64, I32, P]
+            l.oracle_select.argtypes = [P, I64, I64, P]
+            l.oracle_attend.argtypes = [P, P, P, P, I64, I32, P]
+            l.oracle_decode_step.argtypes = [P, P, P, P, P, I32, I32, I32, I64, I32, I32, P, P, P, I32]
+            for f in (l.oracle_rotate, l.oracle_bucket_pack, l.oracle_encode, l.oracle_distance,
+                      l.oracle_select, l.oracle_attend, l.oracle_decode_step):
+                f.restype = ctypes.c_int
+            _lib = l
+        return _lib
+
+
+def _p(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def _check(rc: int, name: str):
+    if rc != 0:
+        raise ValueError(f"oracle: {name} rejected its arguments")
+
+
+def rotate(x_bf16: np.ndarray) -> np.ndarray:
+    """fp32 Hadamard-rotated values of bf16 vectors [..., 128] -> float32 [..., 128]."""
+    x = _c(x_bf16, np.uint16)
+    y = np.empty(x.shape, dtype=np.float32)
+    _check(lib().oracle_rotate(_p(x), x.size // 128, x.shape[-1], _p(y)), "rotate")
+    return y
+
+
+def bucket_pack(y: np.ndarray) -> np.ndarray:
+    """Packed codes of already-rotated fp32 vectors [..., 128] -> uint8 [..., 32]."""
+    y = _c(y, np.float32)
+    out = np.empty(y.shape[:-1] + (32,), dtype=np.uint8)
+    _check(lib().oracle_bucket_pack(_p(y), y.size // 128, y.shape[-1], _p(out)), "bucket_pack")
+    return out
+
+
+def encode(x_bf16: np.ndarray) -> np.ndarray:
+    """Packed 2-bit codes of bf16 vectors [..., 128] -> uint8 [..., 32]."""
+    x = _c(x_bf16, np.uint16)
+    out = np.empty(x.shape[:-1] + (32,), dtype=np.uint8)
+    _check(lib().oracle_encode(_p(x), x.size // 128, x.shape[-1], _p(out)), "encode")
+    return out
+
+
+def distance(qcode: np.ndarray, kcodes: np.ndarray) -> np.ndarray:
+    """L1 distances of one packed query code [32] to packed keys [n, 32] -> int32 [n]."""
+    q = _c(qcode, np.uint8).reshape(32)
+    k = _c(kcodes, np.uint8).reshape(-1, 32)
+    D = np.empty(k.shape[0], dtype=np.int32)
+    _check(lib().oracle_distance(_p(q), _p(k), k.shape[0], 128, _p(D)), "distance")
+    return D
+
+
+def select(D: np.ndarray, k: int) -> np.ndarray:
+    """Token indices of the k smallest (D, index), -1 past len(D) -> int32 [k]."""
+    D = _c(D, np.int32)
+    idx = np.empty(max(k, 1), dtype=np.int32)
+    _check(lib().oracle_select(_p(D), D.size, k, _p(idx)), "select")
+    return idx[:k]
+
+
+def attend(q: np.ndarray, K: np.ndarray, V: np.ndarray, idx: np.ndarray) -> np.ndarray:
+    """float64 attention of one bf16 query [128] over bf16 rows K/V [n, 128] picked by idx."""
+    q = _c(q, np.uint16).reshape(128)
+    K = _c(K, np.uint16).reshape(-1, 128)
+    V = _c(V, np.uint16).reshape(-1, 128)
+    idx = _c(idx, np.int32).reshape(-1)
+    if idx.size and int(idx.max(initial=-1)) >= K.shape[0]:
+        raise ValueError("oracle: idx out of range")
+    out = np.empty(128, dtype=np.float64)
+    _check(lib().oracle_attend(_p(q), _p(K), _p(V), _p(idx), idx.size, 128, _p(out)), "attend")
+    return out
+
+
+def decode_step(q, K, V, codes, seq_lens, budget: int, nthreads: int = 1, want_dist: bool = False):
+    """Whole decode step.  q [B,Hq,128], K/V [B,Hkv,Nmax,128] bf16 bits, codes
+    [B,Hkv,Nmax,32] (from encode), seq_lens int32 [B].
+    Returns (out float64 [B,Hq,128], idx int32 [B,Hq,budget], dist int32 [B,Hq,Nmax] or None)."""
+    q = _c(q, np.uint16)
+    K = _c(K, np.uint16)
+    V = _c(V, np.uint16)
+    codes = _c(codes, np.uint8)
+    lens = _c(seq_lens, np.int32)
+    B, Hq, d = q.shape
+    _, Hkv, Nmax, _ = K.shape
+    if V.shape != K.shape or codes.shape != (B, Hkv, Nmax, 32) or lens.shape != (B,):
+        raise ValueError("oracle: inconsistent shapes")
+    out = np.empty((B, Hq, d), dtype=np.float64)
+    idx = np.empty((B, Hq, max(budget, 1)), dtype=np.int32)
+    dist = np.empty((B, Hq, Nmax), dtype=np.int32) if want_dist else None
+    rc = lib().oracle_decode_step(_p(q), _p(K), _p(V), _p(codes), _p(lens), B, Hq, Hkv, Nmax, d,
+                                  budget, _p(out), _p(idx), _p(dist) if want_dist else None,
+                                  nthreads)
+    _check(rc, "decode_step")
+    return out, idx[:, :, :budget], dist
