@@ -1,0 +1,383 @@
+"""Throughput of the ADAMAS sparse decode path on B200.
+
+One step = one attention layer's decode for the whole batch of the 128K-context
+workload (batch 1, 32 heads, head dim 128, context 131072, budget 1024): append
+one token (its key is encoded into the code cache) and run adamas_decode_step
+(query encode, L1 scoring of all 131072 cached tokens per head, top-1024 select,
+exact attention over the kept rows).  Four layer buffers rotate so that the
+working set (8.5 GiB) is far larger than L2.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Prints one JSON line.  --impl reference times the CPU oracle on a bounded sample
+of the same workload.  Under torchrun every rank runs its own independent copy of
+the workload (weak scaling, no collective on the data path); the time is the max
+over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import glob
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from compressed_sparse_kv_fp32_b200 import accounting, synth  # noqa: E402
+
+METRIC = "decode steps/s and achieved HBM GB/s (% of B200 peak) at 128K ctx, budget 1024"
+UNIT = "decode steps/s"
+WORKLOAD_ID = 3
+BUDGET = 1024
+LAYERS = 4
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", default="adamas", choices=["adamas", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=500)
+    return ap.parse_args()
+
+
+def source_hash() -> str:
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "compressed_sparse_kv_fp32_b200", "csrc", "*"))):
+        h.update(open(f, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        v = float(json.load(open(path))["hbm_gbs"])
+        return v, "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def profiled_traffic(kernel: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on this source."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}.json")
+    try:
+        p = json.load(open(path))
+    except Exception:
+        return None
+    if p.get("source_hash") != source_hash():
+        return None
+    return p.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.rows = []
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append([x.strip() for x in line.split(",")])
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm = [float(r[0]) for r in self.rows if len(r) >= 8 and r[0].replace(".", "").isdigit()]
+        if not sm:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows if len(r) >= 8 for i in range(4)
+                          if r[4 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(self.rows[-1][1]),
+                "samples": len(sm), "reasons": reasons}
+
+
+# ---------------------------------------------------------------- CPU oracle (baseline / reference arm)
+def oracle_sample(w, heads: int, min_seconds: float):
+    """Time the oracle's decode step on `heads` heads of the workload at full context."""
+    from oracle import oracle
+
+    K = np.stack([synth.head_kv(w, 0, h)[0] for h in range(heads)])[None]
+    V = np.stack([synth.head_kv(w, 0, h)[1] for h in range(heads)])[None]
+    q = synth.query(w, 1)[:, :heads]
+    lens = synth.seq_lens(w)
+    codes = oracle.encode(K)
+    cores = os.cpu_count() or 1
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle.decode_step(q, K, V, codes, lens, BUDGET, nthreads=min(cores, heads))
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= min_seconds:
+            break
+    steps = reps * heads / w.Hq
+    return {"value": steps / el, "unit": UNIT, "cores": min(cores, heads), "kind": "oracle",
+            "sample": f"{reps} oracle decode steps over {heads} of {w.Hq} heads at context {w.Nmax}, "
+                      f"budget {BUDGET} (query encode + L1 over every token + sort + float64 attention); "
+                      f"value scaled to whole {w.Hq}-head steps"}
+
+
+def config_block(w):
+    return {"workload": f"{w.name}: batch {w.B}, {w.Hq} heads (MHA), head_dim {w.d}, context {w.Nmax}, "
+                        f"budget {BUDGET}, 1 appended token per step",
+            "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "context": w.Nmax, "budget": BUDGET, "head_dim": w.d,
+            "l2": f"{LAYERS} rotating layer buffers (K, V, codes), working set "
+                  f"{LAYERS * (2 * w.Hkv * w.Nmax * 256 + w.Hkv * w.Nmax * 32) / 2**30:.1f} GiB > L2",
+            "parallelism": "independent replica per GPU"}
+
+
+def run_reference(args, rank, world):
+    w = synth.WORKLOADS[WORKLOAD_ID]
+    if rank != 0:
+        return
+    cb = oracle_sample(w, heads=min(8, os.cpu_count() or 1), min_seconds=15.0)
+    line = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 / cb["value"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u8/f64",
+            "data": "synthetic", "config": config_block(w), "cpu_baseline": cb,
+            "e2e": {"value": cb["value"], "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- GPU arm
+def run_gpu(args, rank, world):
+    import torch
+    import torch.distributed as dist
+
+    from compressed_sparse_kv_fp32_b200 import adamas
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    lib = adamas.load()
+    w = synth.WORKLOADS[WORKLOAD_ID]
+    B, Hq, Hkv, N, d = w.B, w.Hq, w.Hkv, w.Nmax, w.d
+    ctx = N
+
+    # one layer generated on the host, copied into LAYERS device buffers
+    K_host = np.empty((B, Hkv, N, d), dtype=np.uint16)
+    V_host = np.empty_like(K_host)
+    for h in range(Hkv):
+        K_host[0, h], V_host[0, h] = synth.head_kv(w, 0, h)
+
+    def to_dev(a):
+        return torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+
+    layers = []
+    for l in range(LAYERS):
+        K = to_dev(K_host)
+        V = to_dev(V_host)
+        codes = torch.empty((B, Hkv, N, 32), dtype=torch.uint8, device=dev)
+        adamas.encode_keys(K, codes)
+        q = to_dev(synth.query(w, l + 1))
+        out = torch.empty((B, Hq, d), dtype=torch.float32, device=dev)
+        idx = torch.empty((B, Hq, BUDGET), dtype=torch.int32, device=dev)
+        ws = adamas.Workspace(B, Hq, Hkv, N, BUDGET, device=dev)
+        layers.append(dict(K=K, V=V, codes=codes, q=q, out=out, idx=idx, ws=ws))
+    lens = torch.full((B,), ctx, dtype=torch.int32, device=dev)
+    pos = torch.full((B,), ctx - 1, dtype=torch.int32, device=dev)   # the appended token's slot
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.current_stream().cuda_stream
+    calls = []
+    for L in layers:
+        enc = (L["K"].data_ptr(), L["codes"].data_ptr(), pos.data_ptr(), 1, B, Hkv, N, d, stream)
+        dec = (L["q"].data_ptr(), L["codes"].data_ptr(), L["K"].data_ptr(), L["V"].data_ptr(), lens.data_ptr(),
+               B, Hq, Hkv, N, d, BUDGET, L["out"].data_ptr(), L["idx"].data_ptr(), L["ws"].buffer.data_ptr(),
+               L["ws"].nbytes, stream)
+        calls.append((enc, dec))
+    f_enc, f_dec = lib.adamas_encode_keys, lib.adamas_decode_step
+
+    def step(i, ev=None):
+        enc, dec = calls[i % LAYERS]
+        if f_enc(*enc) != 0:
+            raise RuntimeError("encode failed")
+        if ev is not None:
+            ev[0].record()
+        if f_dec(*dec) != 0:
+            raise RuntimeError("decode failed")
+        if ev is not None:
+            ev[1].record()
+
+    gpu_id = "0"
+    try:
+        p = torch.cuda.get_device_properties(dev)
+        gpu_id = f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+    except Exception:
+        gpu_id = str(local)
+    sampler = ClockSampler(gpu_id)
+    sampler.start()
+
+    for i in range(max(3, args.warmup)):
+        step(i)
+    t_end = time.perf_counter() + 1.0          # hold the GPU busy ~1 s so clocks settle
+    i = 0
+    while time.perf_counter() < t_end:
+        step(i)
+        i += 1
+        if i % 256 == 0:
+            torch.cuda.synchronize()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+
+    K_steps = args.steps
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K_steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for i in range(K_steps):
+        step(i, evs[i])
+    t1.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+
+    elapsed_ms = t0.elapsed_time(t1)
+    dec_ms = sum(a.elapsed_time(b) for a, b in evs) / K_steps
+    for L in layers:
+        if L["ws"].device_error() != 0:
+            raise RuntimeError("device error word set during the bench")
+
+    if world > 1:
+        tt = torch.tensor([elapsed_ms, dec_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        elapsed_ms, dec_ms = float(tt[0]), float(tt[1])
+
+    # ---- end to end through the Python API: pinned host inputs in, results out, every step
+    e2e_steps = min(args.e2e_steps, K_steps)
+    q_pin = torch.from_numpy(synth.query(w, 3).view(np.int16)).view(torch.bfloat16).pin_memory()
+    krow_pin = torch.from_numpy(K_host[:, :, ctx - 1].copy().view(np.int16)).view(torch.bfloat16).pin_memory()
+    vrow_pin = torch.from_numpy(V_host[:, :, ctx - 1].copy().view(np.int16)).view(torch.bfloat16).pin_memory()
+    out_pin = torch.empty((B, Hq, d), dtype=torch.float32).pin_memory()
+    idx_pin = torch.empty((B, Hq, BUDGET), dtype=torch.int32).pin_memory()
+    q_dev = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=dev)
+    krow_dev = torch.empty((B, Hkv, d), dtype=torch.bfloat16, device=dev)
+    vrow_dev = torch.empty_like(krow_dev)
+    h2d = q_pin.numel() * 2 + krow_pin.numel() * 2 + vrow_pin.numel() * 2
+    d2h = out_pin.numel() * 4 + idx_pin.numel() * 4
+
+    def e2e_step(i):
+        L = layers[i % LAYERS]
+        q_dev.copy_(q_pin, non_blocking=True)
+        krow_dev.copy_(krow_pin, non_blocking=True)
+        vrow_dev.copy_(vrow_pin, non_blocking=True)
+        L["K"][:, :, ctx - 1].copy_(krow_dev)
+        L["V"][:, :, ctx - 1].copy_(vrow_dev)
+        adamas.encode_keys(L["K"], L["codes"], pos, 1)
+        adamas.decode_step(q_dev, L["codes"], L["K"], L["V"], lens, BUDGET, L["ws"], L["out"], L["idx"])
+        out_pin.copy_(L["out"], non_blocking=True)
+        idx_pin.copy_(L["idx"], non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+
+    for i in range(3):
+        e2e_step(i)
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(e2e_steps):
+        e2e_step(i)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        tt = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt[0])
+
+    if rank != 0:
+        return
+    ms_per_step = elapsed_ms / K_steps
+    value = world * K_steps / (elapsed_ms / 1e3)
+    step_bytes = accounting.decode_step_bytes([ctx] * B, Hq, Hkv, BUDGET, d)
+    enc_bytes = B * Hkv * accounting.encode_bytes_per_vector(d)
+    peak, peak_kind = measured_peak()
+    achieved_dec = step_bytes["total"] / (dec_ms / 1e3) / 1e9
+    achieved_step = (step_bytes["total"] + enc_bytes) / (ms_per_step / 1e3) / 1e9
+    traffic = profiled_traffic("decode_step_kernel_mha32_128k")
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K_steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "u8/fp32", "data": "synthetic",
+        "config": config_block(w),
+        "achieved_hbm_gbs": achieved_step, "pct_of_peak_hbm": 100.0 * achieved_step / peak,
+        "peak_hbm_gbs": peak, "peak_kind": peak_kind,
+        "roofline": {"bound": "hbm", "kernel": "decode_step_kernel", "achieved": achieved_dec, "peak": peak,
+                     "unit": "GB/s", "frac": achieved_dec / peak, "traffic": traffic,
+                     "algorithmic_bytes_per_launch": step_bytes["total"], "avg_launch_us": dec_ms * 1e3,
+                     "peak_source": f"MEASURED_PEAKS.json hbm_gbs ({peak_kind})"},
+        "e2e": {"value": world * e2e_steps / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": 2 * K_steps,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = oracle_sample(w, heads=min(8, os.cpu_count() or 1), min_seconds=12.0)
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_gpu(args, rank, world)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,194 @@
+"""Python binding of libadamas.so (C ABI in include/adamas.h).
+
+Argument marshalling only: every step of the method runs in the library's CUDA
+kernels.  Tensors are torch CUDA tensors; calls are enqueued on the current torch
+stream.  The library must have been built (compressed_sparse_kv_fp32_b200.build);
+there is no fallback of any kind.
+
+Method: ADAMAS long-context sparse attention article (lnwmold.com/news/826806),
+§2.1 Hadamard rotation, §2.2 dynamic 2-bit bucketing, §3.1 packed code cache,
+§2.3 Manhattan-distance scoring, §5.2 token budget.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional, Tuple
+
+import torch
+
+from .build import LIBRARY
+
+HEAD_DIM = 128
+DEVERR_SEQLEN = 0x1
+DEVERR_TIMEOUT = 0x2
+
+_lock = threading.Lock()
+_lib = None
+
+SYMBOLS = (
+    "adamas_status_string", "adamas_version", "adamas_workspace_bytes", "adamas_workspace_init",
+    "adamas_encode_keys", "adamas_decode_step", "adamas_score", "adamas_get_device_error",
+)
+
+
+class AdamasError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} ({status})")
+
+
+def load(path: str = LIBRARY) -> ctypes.CDLL:
+    """Load libadamas.so and declare its signatures (raises if it was not built)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(path):
+            raise ImportError(f"{path} is missing: build it with `python -m compressed_sparse_kv_fp32_b200.build`")
+        l = ctypes.CDLL(path)
+        P, I, I64, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+        l.adamas_status_string.argtypes = [I]
+        l.adamas_status_string.restype = ctypes.c_char_p
+        l.adamas_version.argtypes = []
+        l.adamas_version.restype = I
+        l.adamas_workspace_bytes.argtypes = [I, I, I, I64, I, I]
+        l.adamas_workspace_bytes.restype = SZ
+        l.adamas_workspace_init.argtypes = [P, SZ, P]
+        l.adamas_workspace_init.restype = I
+        l.adamas_encode_keys.argtypes = [P, P, P, I, I, I, I64, I, P]
+        l.adamas_encode_keys.restype = I
+        l.adamas_decode_step.argtypes = [P, P, P, P, P, I, I, I, I64, I, I, P, P, P, SZ, P]
+        l.adamas_decode_step.restype = I
+        l.adamas_score.argtypes = [P, P, P, I, I, I, I64, I, P, P]
+        l.adamas_score.restype = I
+        l.adamas_get_device_error.argtypes = [P, SZ, ctypes.POINTER(ctypes.c_uint32), P]
+        l.adamas_get_device_error.restype = I
+        _lib = l
+        return l
+
+
+def status_string(status: int) -> str:
+    return load().adamas_status_string(int(status)).decode()
+
+
+def _check(rc: int, where: str):
+    if rc != 0:
+        raise AdamasError(rc, where)
+
+
+def _stream(stream: Optional[torch.cuda.Stream]) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _need(t: torch.Tensor, name: str, dtype: torch.dtype, shape: Optional[tuple] = None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be on a CUDA device")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def workspace_bytes(B: int, Hq: int, Hkv: int, Nmax: int, budget: int, d: int = HEAD_DIM) -> int:
+    n = load().adamas_workspace_bytes(B, Hq, Hkv, Nmax, d, budget)
+    if n == 0:
+        raise AdamasError(-2, "adamas_workspace_bytes")
+    return int(n)
+
+
+class Workspace:
+    """Device workspace of adamas_decode_step, zero-filled on creation."""
+
+    def __init__(self, B: int, Hq: int, Hkv: int, Nmax: int, budget: int, device=None,
+                 stream: Optional[torch.cuda.Stream] = None):
+        self.nbytes = workspace_bytes(B, Hq, Hkv, Nmax, budget)
+        self.buffer = torch.empty(self.nbytes, dtype=torch.uint8,
+                                  device=device if device is not None else "cuda")
+        self.reset(stream)
+
+    def reset(self, stream: Optional[torch.cuda.Stream] = None):
+        _check(load().adamas_workspace_init(self.buffer.data_ptr(), self.nbytes, _stream(stream)),
+               "adamas_workspace_init")
+
+    def device_error(self, stream: Optional[torch.cuda.Stream] = None) -> int:
+        """Synchronise the stream and return the device error word (DEVERR_* bits)."""
+        word = ctypes.c_uint32(0)
+        rc = load().adamas_get_device_error(self.buffer.data_ptr(), self.nbytes, ctypes.byref(word),
+                                            _stream(stream))
+        if rc not in (0, -5):
+            raise AdamasError(rc, "adamas_get_device_error")
+        return int(word.value)
+
+
+def encode_keys(K: torch.Tensor, codes: torch.Tensor, pos_begin: Optional[torch.Tensor] = None,
+                count: Optional[int] = None, stream: Optional[torch.cuda.Stream] = None):
+    """Encode K [B,Hkv,Nmax,128] bf16 into codes [B,Hkv,Nmax,32] uint8 at positions
+    [pos_begin[b], pos_begin[b] + count) (all positions by default)."""
+    _need(K, "K", torch.bfloat16)
+    if K.dim() != 4 or K.shape[-1] != HEAD_DIM:
+        raise ValueError("K must be [B, Hkv, Nmax, 128]")
+    B, Hkv, Nmax, d = K.shape
+    _need(codes, "codes", torch.uint8, (B, Hkv, Nmax, d // 4))
+    if pos_begin is not None:
+        _need(pos_begin, "pos_begin", torch.int32, (B,))
+    n = Nmax if count is None else int(count)
+    _check(load().adamas_encode_keys(K.data_ptr(), codes.data_ptr(), _ptr(pos_begin), n, B, Hkv, Nmax, d,
+                                     _stream(stream)), "adamas_encode_keys")
+    return codes
+
+
+def decode_step(q: torch.Tensor, codes: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
+                seq_lens: torch.Tensor, budget: int, workspace: Workspace,
+                out: Optional[torch.Tensor] = None, idx: Optional[torch.Tensor] = None,
+                stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """One decode step: returns (out [B,Hq,128] fp32, idx [B,Hq,budget] int32)."""
+    _need(q, "q", torch.bfloat16)
+    if q.dim() != 3:
+        raise ValueError("q must be [B, Hq, 128]")
+    B, Hq, d = q.shape
+    _need(K, "K", torch.bfloat16)
+    if K.dim() != 4:
+        raise ValueError("K must be [B, Hkv, Nmax, 128]")
+    _, Hkv, Nmax, _ = K.shape
+    _need(K, "K", torch.bfloat16, (B, Hkv, Nmax, d))
+    _need(V, "V", torch.bfloat16, (B, Hkv, Nmax, d))
+    _need(codes, "codes", torch.uint8, (B, Hkv, Nmax, d // 4))
+    _need(seq_lens, "seq_lens", torch.int32, (B,))
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)
+    if idx is None:
+        idx = torch.empty((B, Hq, budget), dtype=torch.int32, device=q.device)
+    _need(out, "out", torch.float32, (B, Hq, d))
+    _need(idx, "idx", torch.int32, (B, Hq, budget))
+    rc = load().adamas_decode_step(q.data_ptr(), codes.data_ptr(), K.data_ptr(), V.data_ptr(),
+                                   seq_lens.data_ptr(), B, Hq, Hkv, Nmax, d, budget, out.data_ptr(),
+                                   idx.data_ptr() if budget > 0 else None,
+                                   workspace.buffer.data_ptr(), workspace.nbytes, _stream(stream))
+    _check(rc, "adamas_decode_step")
+    return out, idx
+
+
+def score(q: torch.Tensor, codes: torch.Tensor, seq_lens: torch.Tensor, Hkv: Optional[int] = None,
+          stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """L1 code distances [B,Hq,Nmax] (uint16 values in an int16 tensor; 0xFFFF past each length)."""
+    _need(q, "q", torch.bfloat16)
+    B, Hq, d = q.shape
+    _need(codes, "codes", torch.uint8)
+    _, Hkv, Nmax, _ = codes.shape
+    _need(codes, "codes", torch.uint8, (B, Hkv, Nmax, d // 4))
+    _need(seq_lens, "seq_lens", torch.int32, (B,))
+    dist = torch.empty((B, Hq, Nmax), dtype=torch.int16, device=q.device)
+    _check(load().adamas_score(q.data_ptr(), codes.data_ptr(), seq_lens.data_ptr(), B, Hq, Hkv, Nmax, d,
+                               dist.data_ptr(), _stream(stream)), "adamas_score")
+    return dist

@@ -1,0 +1,356 @@
+// C ABI of the ADAMAS sparse decode library (declared in include/adamas.h):
+// argument checks, workspace layout, and the launches of the sm_100a kernels.
+//
+// Method: ADAMAS long-context sparse attention article (lnwmold.com/news/826806),
+// §2.1 Hadamard rotation, §2.2 dynamic 2-bit bucketing, §3.1 packed code cache,
+// §2.3 Manhattan-distance scoring, §5.2 token budget.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/adamas.h"
+#include "common.cuh"
+#include "decode.cuh"
+#include "encode.cuh"
+#include "score.cuh"
+
+namespace adamas {
+
+// ------------------------------------------------------------------ key encoder
+constexpr int kEncThreads = 128;       // one vector per thread, one tile of 128 positions per block
+constexpr int kEncRowWords = 68;       // 64 words of bf16 + 4 words of padding (bank spread)
+
+__global__ void __launch_bounds__(kEncThreads) encode_keys_kernel(const uint16_t* __restrict__ K,
+                                                                  uint8_t* __restrict__ codes,
+                                                                  const int32_t* __restrict__ pos_begin,
+                                                                  int count, int Hkv, int64_t Nmax) {
+  __shared__ __align__(16) uint32_t tile[kEncThreads * kEncRowWords];
+  const int tid = threadIdx.x;
+  const int hk = blockIdx.y;
+  const int b = hk / Hkv;
+  const int64_t p0 = pos_begin ? (int64_t)pos_begin[b] : 0;
+  const int64_t first = (int64_t)blockIdx.x * kEncThreads;
+  const uint16_t* kbase = K + (int64_t)hk * Nmax * kDim;
+
+  // coalesced 16-byte loads of the tile's rows into padded shared memory
+#pragma unroll 4
+  for (int i = tid; i < kEncThreads * 16; i += kEncThreads) {
+    const int row = i >> 4, ch = i & 15;
+    const int64_t r = first + row, pos = p0 + r;
+    if (r < count && pos >= 0 && pos < Nmax) {
+      const uint4 v = *reinterpret_cast<const uint4*>(kbase + pos * kDim + ch * 8);
+      *reinterpret_cast<uint4*>(&tile[row * kEncRowWords + ch * 4]) = v;
+    }
+  }
+  __syncthreads();
+
+  const int64_t r = first + tid, pos = p0 + r;
+  if (r >= count || pos < 0 || pos >= Nmax) return;
+  float v[kDim];
+#pragma unroll
+  for (int ch = 0; ch < 16; ++ch) {
+    const uint4 w = *reinterpret_cast<const uint4*>(&tile[tid * kEncRowWords + ch * 4]);
+    v[8 * ch + 0] = bf16_lo(w.x); v[8 * ch + 1] = bf16_hi(w.x);
+    v[8 * ch + 2] = bf16_lo(w.y); v[8 * ch + 3] = bf16_hi(w.y);
+    v[8 * ch + 4] = bf16_lo(w.z); v[8 * ch + 5] = bf16_hi(w.z);
+    v[8 * ch + 6] = bf16_lo(w.w); v[8 * ch + 7] = bf16_hi(w.w);
+  }
+  fwht128_thread(v);
+  uint32_t w[kCodeWords];
+  bucket_pack_thread(v, w);
+  uint4* dst = reinterpret_cast<uint4*>(codes + ((int64_t)hk * Nmax + pos) * kCodeBytes);
+  dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+  dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+}
+
+// ------------------------------------------------------------------ distance dump (test entry point)
+constexpr int kScoreThreads = 256;
+constexpr int kScoreUnroll = 4;
+
+template <int G>
+__global__ void __launch_bounds__(kScoreThreads) score_kernel(const uint16_t* __restrict__ q,
+                                                              const uint8_t* __restrict__ codes,
+                                                              const int32_t* __restrict__ seq_lens, int Hq,
+                                                              int Hkv, int64_t Nmax, uint16_t* __restrict__ dist) {
+  __shared__ uint32_t sq[G * kCodeWords];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int hk = blockIdx.y, b = hk / Hkv, kvh = hk - b * Hkv;
+  if (warp < G) {
+    const uint32_t w = encode128_warp(q + ((int64_t)b * Hq + kvh * G + warp) * kDim, lane);
+    if (lane < kCodeWords) sq[warp * kCodeWords + lane] = w;
+  }
+  __syncthreads();
+  int64_t len = seq_lens[b];
+  len = len < 0 ? 0 : (len > Nmax ? Nmax : len);
+  uint32_t qw[G][kCodeWords];
+#pragma unroll
+  for (int g = 0; g < G; ++g)
+#pragma unroll
+    for (int w = 0; w < kCodeWords; ++w) qw[g][w] = sq[g * kCodeWords + w];
+  const int64_t first = (int64_t)blockIdx.x * kScoreThreads * kScoreUnroll;
+#pragma unroll
+  for (int j = 0; j < kScoreUnroll; ++j) {
+    const int64_t t = first + (int64_t)j * kScoreThreads + tid;
+    if (t >= Nmax) break;
+    uint32_t kc[kCodeWords], e[kCodeWords];
+    if (t < len) {
+      ld_stream_v8(codes + ((int64_t)hk * Nmax + t) * kCodeBytes, kc);
+      key_odd_mask(kc, e);
+    }
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const uint16_t d = t < len ? (uint16_t)l1_distance(kc, e, qw[g]) : (uint16_t)0xFFFF;
+      dist[((int64_t)b * Hq + kvh * G + g) * Nmax + t] = d;
+    }
+  }
+}
+
+// ------------------------------------------------------------------ host side
+struct DeviceInfo {
+  int sms = 0;
+  size_t smem_optin = 0;
+  bool attrs_set[kMaxGroup + 1] = {};
+};
+
+static std::mutex g_mutex;
+static DeviceInfo g_devices[64];
+
+static int device_info(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ADAMAS_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceInfo& d = g_devices[dev];
+  if (d.sms == 0) {
+    int sms = 0, optin = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+      return ADAMAS_ERR_CUDA;
+    d.smem_optin = (size_t)optin;
+    d.sms = sms;
+  }
+  *out = &d;
+  return ADAMAS_OK;
+}
+
+struct WsLayout {
+  size_t ctrl, head_done, hist, partial, dspill, total;
+  int S;
+  int64_t range_cap;
+  bool smem_d;
+  size_t smem;
+};
+
+static size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+static int check_shape(int B, int Hq, int Hkv, int64_t Nmax, int d, int budget) {
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || Nmax < 0 || budget < 0) return ADAMAS_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return ADAMAS_ERR_INVALID_ARG;
+  if (d != kDim) return ADAMAS_ERR_UNSUPPORTED;
+  if (Hq / Hkv > kMaxGroup || B > kMaxBatch || Nmax > INT32_MAX) return ADAMAS_ERR_UNSUPPORTED;
+  if ((int64_t)B * Hkv > 65535) return ADAMAS_ERR_UNSUPPORTED;
+  return ADAMAS_OK;
+}
+
+static int ws_layout(int B, int Hq, int Hkv, int64_t Nmax, int budget, const DeviceInfo& dev, WsLayout* L) {
+  (void)budget;
+  const int G = Hq / Hkv;
+  const int64_t umax = (int64_t)B * Hkv * Nmax;
+  int64_t want = (umax + 2047) / 2048;
+  L->S = (int)(want < 1 ? 1 : (want > dev.sms ? dev.sms : want));
+  L->range_cap = umax > 0 ? (umax + L->S - 1) / L->S : 1;
+  L->smem_d = DecodeSmem::total(B, G, L->range_cap, true) <= dev.smem_optin;
+  L->smem = DecodeSmem::total(B, G, L->range_cap, L->smem_d);
+  if (L->smem > dev.smem_optin) return ADAMAS_ERR_UNSUPPORTED;
+  size_t off = 0;
+  L->ctrl = off;      off += align256(64 * sizeof(uint32_t));
+  L->head_done = off; off += align256((size_t)B * Hq * sizeof(uint32_t));
+  L->hist = off;      off += align256((size_t)(L->S + B * Hkv) * G * kHistStride * sizeof(uint32_t));
+  L->partial = off;   off += align256((size_t)(L->S + B * Hq) * kPartial * sizeof(float));
+  L->dspill = off;    off += L->smem_d ? 0 : align256((size_t)L->S * G * L->range_cap * sizeof(uint16_t));
+  L->total = off;
+  return ADAMAS_OK;
+}
+
+static bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+template <int G>
+static int launch_decode(const DecodeParams& prm, const WsLayout& L, DeviceInfo& dev, cudaStream_t stream) {
+  auto kernel = decode_step_kernel<G>;
+  {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (!dev.attrs_set[G]) {
+      if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dev.smem_optin) !=
+          cudaSuccess)
+        return ADAMAS_ERR_CUDA;
+      dev.attrs_set[G] = true;
+    }
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)L.S);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = L.smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kernel, prm) != cudaSuccess) return ADAMAS_ERR_CUDA;
+  return ADAMAS_OK;
+}
+
+template <int G>
+static void launch_score(dim3 grid, cudaStream_t st, const uint16_t* q, const uint8_t* codes, const int32_t* lens,
+                         int Hq, int Hkv, int64_t Nmax, uint16_t* dist) {
+  score_kernel<G><<<grid, kScoreThreads, 0, st>>>(q, codes, lens, Hq, Hkv, Nmax, dist);
+}
+
+}  // namespace adamas
+
+using namespace adamas;
+
+extern "C" {
+
+const char* adamas_status_string(int status) {
+  switch (status) {
+    case ADAMAS_OK: return "ok";
+    case ADAMAS_ERR_INVALID_ARG: return "invalid argument";
+    case ADAMAS_ERR_UNSUPPORTED: return "unsupported size or configuration";
+    case ADAMAS_ERR_WORKSPACE: return "workspace missing or too small";
+    case ADAMAS_ERR_CUDA: return "CUDA runtime error";
+    case ADAMAS_ERR_DEVICE: return "device error word set";
+    default: return "unknown status";
+  }
+}
+
+int adamas_version(void) { return 100; }
+
+size_t adamas_workspace_bytes(int B, int Hq, int Hkv, int64_t Nmax, int d, int budget) {
+  if (check_shape(B, Hq, Hkv, Nmax, d, budget) != ADAMAS_OK) return 0;
+  DeviceInfo* dev = nullptr;
+  if (device_info(&dev) != ADAMAS_OK) return 0;
+  WsLayout L;
+  if (ws_layout(B, Hq, Hkv, Nmax, budget, *dev, &L) != ADAMAS_OK) return 0;
+  return L.total;
+}
+
+int adamas_workspace_init(void* workspace, size_t workspace_bytes, adamas_stream_t stream) {
+  if (!workspace || workspace_bytes == 0) return ADAMAS_ERR_INVALID_ARG;
+  if (cudaMemsetAsync(workspace, 0, workspace_bytes, (cudaStream_t)stream) != cudaSuccess) return ADAMAS_ERR_CUDA;
+  return ADAMAS_OK;
+}
+
+int adamas_encode_keys(const void* K, uint8_t* codes, const int32_t* pos_begin, int count, int B, int Hkv,
+                       int64_t Nmax, int d, adamas_stream_t stream) {
+  const int rc = check_shape(B, Hkv, Hkv, Nmax, d, 0);
+  if (rc != ADAMAS_OK) return rc;
+  if (count < 0) return ADAMAS_ERR_INVALID_ARG;
+  if (B == 0 || count == 0 || Nmax == 0) return ADAMAS_OK;
+  if (!K || !codes || !aligned(K, 16) || !aligned(codes, 32)) return ADAMAS_ERR_INVALID_ARG;
+  if (pos_begin && !aligned(pos_begin, 4)) return ADAMAS_ERR_INVALID_ARG;
+  const dim3 grid((unsigned)((count + kEncThreads - 1) / kEncThreads), (unsigned)(B * Hkv));
+  encode_keys_kernel<<<grid, kEncThreads, 0, (cudaStream_t)stream>>>(
+      static_cast<const uint16_t*>(K), codes, pos_begin, count, Hkv, Nmax);
+  if (cudaGetLastError() != cudaSuccess) return ADAMAS_ERR_CUDA;
+  return ADAMAS_OK;
+}
+
+int adamas_decode_step(const void* q, const uint8_t* codes, const void* K, const void* V, const int32_t* seq_lens,
+                       int B, int Hq, int Hkv, int64_t Nmax, int d, int budget, float* out, int32_t* idx,
+                       void* workspace, size_t workspace_bytes, adamas_stream_t stream) {
+  int rc = check_shape(B, Hq, Hkv, Nmax, d, budget);
+  if (rc != ADAMAS_OK) return rc;
+  if (B == 0) return ADAMAS_OK;
+  if (!q || !seq_lens || !out || (budget > 0 && !idx)) return ADAMAS_ERR_INVALID_ARG;
+  if (Nmax > 0 && (!codes || !K || !V)) return ADAMAS_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(codes, 32) || !aligned(K, 16) || !aligned(V, 16) || !aligned(out, 16) ||
+      !aligned(idx, 4) || !aligned(seq_lens, 4))
+    return ADAMAS_ERR_INVALID_ARG;
+  DeviceInfo* dev = nullptr;
+  if ((rc = device_info(&dev)) != ADAMAS_OK) return rc;
+  WsLayout L;
+  if ((rc = ws_layout(B, Hq, Hkv, Nmax, budget, *dev, &L)) != ADAMAS_OK) return rc;
+  if (!workspace || workspace_bytes < L.total || !aligned(workspace, 16)) return ADAMAS_ERR_WORKSPACE;
+
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  DecodeParams prm;
+  prm.q = static_cast<const uint16_t*>(q);
+  prm.codes = codes;
+  prm.K = static_cast<const uint16_t*>(K);
+  prm.V = static_cast<const uint16_t*>(V);
+  prm.seq_lens = seq_lens;
+  prm.out = out;
+  prm.idx = idx;
+  prm.ctrl = reinterpret_cast<uint32_t*>(ws + L.ctrl);
+  prm.head_done = reinterpret_cast<uint32_t*>(ws + L.head_done);
+  prm.hist = reinterpret_cast<uint32_t*>(ws + L.hist);
+  prm.partial = reinterpret_cast<float*>(ws + L.partial);
+  prm.dglobal = L.smem_d ? nullptr : reinterpret_cast<uint16_t*>(ws + L.dspill);
+  prm.B = B;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.Nmax = Nmax;
+  prm.budget = budget;
+  prm.S = L.S;
+  prm.range_cap = L.range_cap;
+  prm.smem_d = L.smem_d ? 1 : 0;
+
+  cudaStream_t st = (cudaStream_t)stream;
+  switch (Hq / Hkv) {
+    case 1: rc = launch_decode<1>(prm, L, *dev, st); break;
+    case 2: rc = launch_decode<2>(prm, L, *dev, st); break;
+    case 3: rc = launch_decode<3>(prm, L, *dev, st); break;
+    case 4: rc = launch_decode<4>(prm, L, *dev, st); break;
+    case 5: rc = launch_decode<5>(prm, L, *dev, st); break;
+    case 6: rc = launch_decode<6>(prm, L, *dev, st); break;
+    case 7: rc = launch_decode<7>(prm, L, *dev, st); break;
+    case 8: rc = launch_decode<8>(prm, L, *dev, st); break;
+    default: rc = ADAMAS_ERR_UNSUPPORTED;
+  }
+  if (rc == ADAMAS_OK && cudaGetLastError() != cudaSuccess) rc = ADAMAS_ERR_CUDA;
+  return rc;
+}
+
+int adamas_score(const void* q, const uint8_t* codes, const int32_t* seq_lens, int B, int Hq, int Hkv, int64_t Nmax,
+                 int d, uint16_t* dist, adamas_stream_t stream) {
+  const int rc = check_shape(B, Hq, Hkv, Nmax, d, 0);
+  if (rc != ADAMAS_OK) return rc;
+  if (B == 0 || Nmax == 0) return ADAMAS_OK;
+  if (!q || !codes || !seq_lens || !dist) return ADAMAS_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(codes, 32) || !aligned(seq_lens, 4) || !aligned(dist, 2))
+    return ADAMAS_ERR_INVALID_ARG;
+  const int64_t per_block = (int64_t)kScoreThreads * kScoreUnroll;
+  const dim3 grid((unsigned)((Nmax + per_block - 1) / per_block), (unsigned)(B * Hkv));
+  cudaStream_t st = (cudaStream_t)stream;
+  const uint16_t* qq = static_cast<const uint16_t*>(q);
+  switch (Hq / Hkv) {
+    case 1: launch_score<1>(grid, st, qq, codes, seq_lens, Hq, Hkv, Nmax, dist); break;
+    case 2: launch_score<2>(grid, st, qq, codes, seq_lens, Hq, Hkv, Nmax, dist); break;
+    case 3: launch_score<3>(grid, st, qq, codes, seq_lens, Hq, Hkv, Nmax, dist); break;
+    case 4: launch_score<4>(grid, st, qq, codes, seq_lens, Hq, Hkv, Nmax, dist); break;
+    case 5: launch_score<5>(grid, st, qq, codes, seq_lens, Hq, Hkv, Nmax, dist); break;
+    case 6: launch_score<6>(grid, st, qq, codes, seq_lens, Hq, Hkv, Nmax, dist); break;
+    case 7: launch_score<7>(grid, st, qq, codes, seq_lens, Hq, Hkv, Nmax, dist); break;
+    case 8: launch_score<8>(grid, st, qq, codes, seq_lens, Hq, Hkv, Nmax, dist); break;
+    default: return ADAMAS_ERR_UNSUPPORTED;
+  }
+  if (cudaGetLastError() != cudaSuccess) return ADAMAS_ERR_CUDA;
+  return ADAMAS_OK;
+}
+
+int adamas_get_device_error(const void* workspace, size_t workspace_bytes, uint32_t* error_word,
+                            adamas_stream_t stream) {
+  if (!workspace || !error_word || workspace_bytes < 64 * sizeof(uint32_t)) return ADAMAS_ERR_INVALID_ARG;
+  uint32_t word = 0;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (cudaMemcpyAsync(&word, static_cast<const uint32_t*>(workspace) + 2, sizeof word, cudaMemcpyDeviceToHost, st) !=
+          cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return ADAMAS_ERR_CUDA;
+  *error_word = word;
+  return word == 0 ? ADAMAS_OK : ADAMAS_ERR_DEVICE;
+}
+
+}  // extern "C"

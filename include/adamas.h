@@ -1,0 +1,147 @@
+/*
+ * adamas.h -- C ABI of the B200 (sm_100a) ADAMAS sparse decode attention library.
+ *
+ * The method is the one described in the ADAMAS long-context sparse attention
+ * article (lnwmold.com/news/826806):
+ *   §2.1  queries and cached keys are rotated by an orthogonal Hadamard matrix,
+ *         which leaves every q.k unchanged and spreads outlier channels;
+ *   §2.2  each rotated vector is bucketed into 2-bit codes by three dynamic
+ *         thresholds (-m/2, 0, +m/2), m = max |y| over the 128-dim group;
+ *   §3.1  the codes are kept as a packed cache, four codes per byte;
+ *   §2.3  every cached token is scored by the Manhattan (L1) distance between
+ *         its codes and the query's codes (a smaller distance is more relevant);
+ *   §5.2  only a token budget of the best-scoring tokens is kept, and exact
+ *         softmax attention runs over the K/V rows of those tokens.
+ *
+ * Conventions shared by every entry point
+ *   - Head dimension d must be 128 (one bucketing group per vector).
+ *   - Tensors are dense row-major in device memory:
+ *       q       [B][Hq][128]          bf16
+ *       K, V    [B][Hkv][Nmax][128]   bf16
+ *       codes   [B][Hkv][Nmax][32]    uint8, four 2-bit codes per byte, the code of
+ *                                     dimension 4j in bits 7:6 of byte j
+ *       out     [B][Hq][128]          fp32
+ *       idx     [B][Hq][budget]       int32
+ *     Query head h reads kv head h / (Hq / Hkv) (grouped-query attention).
+ *   - The caller owns every buffer and the stream.  Calls only enqueue work on
+ *     `stream` (a cudaStream_t; NULL is the legacy default stream) and return;
+ *     they never allocate, free or synchronise, except adamas_get_device_error,
+ *     which synchronises `stream` to read the error word.
+ *   - codes must be 32-byte aligned (it is streamed with 32-byte loads); the
+ *     other bf16/fp32 tensors and the workspace 16-byte aligned; int32 arrays
+ *     4-byte aligned.  Inputs must be finite: NaN or Inf in q or K gives
+ *     unspecified codes, indices and outputs (never an out-of-bounds access).
+ *   - Argument errors are detected on the host before anything is enqueued and
+ *     are returned as a negative status; nothing is written in that case.  A
+ *     failed launch returns ADAMAS_ERR_CUDA.  Conditions only the GPU can see
+ *     (a sequence length outside [0, Nmax], a cross-block wait that timed out)
+ *     set bits of an error word in the workspace; see adamas_get_device_error.
+ *   - No exception crosses this interface.  All entry points are thread-safe
+ *     for distinct workspaces.
+ */
+#ifndef ADAMAS_H
+#define ADAMAS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* cudaStream_t without including the CUDA runtime headers */
+typedef struct CUstream_st *adamas_stream_t;
+
+enum adamas_status {
+    ADAMAS_OK = 0,
+    ADAMAS_ERR_INVALID_ARG = -1, /* null/misaligned pointer, bad size or shape */
+    ADAMAS_ERR_UNSUPPORTED = -2, /* d != 128, group size > 8, batch > 1024, ... */
+    ADAMAS_ERR_WORKSPACE = -3,   /* workspace missing or smaller than adamas_workspace_bytes */
+    ADAMAS_ERR_CUDA = -4,        /* a CUDA runtime call or kernel launch failed */
+    ADAMAS_ERR_DEVICE = -5       /* the device error word is non-zero */
+};
+
+/* Bits of the device error word. */
+#define ADAMAS_DEVERR_SEQLEN 0x1u  /* a seq_lens entry was outside [0, Nmax]; it was clamped */
+#define ADAMAS_DEVERR_TIMEOUT 0x2u /* a grid-wide wait gave up; the step's outputs are invalid */
+
+/* Static description of a status code (never NULL). */
+const char *adamas_status_string(int status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int adamas_version(void);
+
+/*
+ * Bytes of device workspace adamas_decode_step needs for these sizes on the
+ * current CUDA device (0 when the sizes are unsupported).  The workspace holds
+ * per-block token histograms, partial softmax states, grid-wait counters and
+ * the error word.  It must be zero-filled once before its first use
+ * (adamas_workspace_init); every step leaves it ready for the next one.  One
+ * workspace must not be used by two steps that may run concurrently.
+ */
+size_t adamas_workspace_bytes(int B, int Hq, int Hkv, int64_t Nmax, int d, int budget);
+
+/* Zero-fill a workspace on `stream` (asynchronous).  Also the way to clear the
+ * error word and recover after ADAMAS_DEVERR_TIMEOUT. */
+int adamas_workspace_init(void *workspace, size_t workspace_bytes, adamas_stream_t stream);
+
+/*
+ * Encode cached keys into packed 2-bit codes (article §2.1 rotation, §2.2
+ * bucketing, §3.1 packing).  For every (b, kv head) it encodes positions
+ * [p, p + count) with p = pos_begin[b] (pos_begin: device int32[B], or NULL for
+ * p = 0); positions outside [0, Nmax) are skipped.  Use count = Nmax at prefill
+ * and count = 1 with pos_begin = the new token's position when appending.
+ *   K      device bf16 [B][Hkv][Nmax][128]  (read)
+ *   codes  device uint8 [B][Hkv][Nmax][32]  (written at the encoded positions)
+ * The rotation is an fp32 Sylvester-order butterfly (stage widths 1..64, no
+ * fused multiply-add) followed by one multiply by RN(1/sqrt(128)); the codes are
+ * bit-identical to the CPU oracle's.
+ */
+int adamas_encode_keys(const void *K, uint8_t *codes, const int32_t *pos_begin, int count, int B,
+                       int Hkv, int64_t Nmax, int d, adamas_stream_t stream);
+
+/*
+ * One decode step of one attention layer for the whole batch: encode q, score
+ * every cached token t < seq_lens[b] of the query head's kv head by the L1
+ * distance D of the codes (article §2.3), keep k_eff = min(budget, seq_lens[b])
+ * tokens of smallest (D, t) -- ties go to the lower token index -- and run exact
+ * softmax attention with scale 1/sqrt(128) over their bf16 K/V rows, in fp32.
+ *   q         device bf16 [B][Hq][128]
+ *   codes     device uint8 [B][Hkv][Nmax][32]  (from adamas_encode_keys)
+ *   K, V      device bf16 [B][Hkv][Nmax][128]
+ *   seq_lens  device int32 [B]
+ *   out       device fp32 [B][Hq][128]   softmax-weighted sum of the kept V rows
+ *                                        (0 when k_eff = 0)
+ *   idx       device int32 [B][Hq][budget]  kept token positions in (D, t)
+ *                                        order, -1 past k_eff
+ *   workspace device, >= adamas_workspace_bytes(...) bytes, zero-filled once
+ * The step runs as one cooperative kernel with one block per SM.
+ */
+int adamas_decode_step(const void *q, const uint8_t *codes, const void *K, const void *V,
+                       const int32_t *seq_lens, int B, int Hq, int Hkv, int64_t Nmax, int d,
+                       int budget, float *out, int32_t *idx, void *workspace,
+                       size_t workspace_bytes, adamas_stream_t stream);
+
+/*
+ * Debug and test entry point: the distances the decode step ranks by.
+ *   dist  device uint16 [B][Hq][Nmax]: D in [0, 384] for t < seq_lens[b],
+ *         0xFFFF past the sequence length.
+ * Same argument rules as adamas_decode_step; seq_lens outside [0, Nmax] are
+ * clamped (no error word here).
+ */
+int adamas_score(const void *q, const uint8_t *codes, const int32_t *seq_lens, int B, int Hq,
+                 int Hkv, int64_t Nmax, int d, uint16_t *dist, adamas_stream_t stream);
+
+/*
+ * Synchronise `stream`, then copy the workspace's device error word into
+ * *error_word (ADAMAS_DEVERR_* bits).  Returns ADAMAS_OK when the word is zero,
+ * ADAMAS_ERR_DEVICE when it is not.
+ */
+int adamas_get_device_error(const void *workspace, size_t workspace_bytes, uint32_t *error_word,
+                            adamas_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ADAMAS_H */
