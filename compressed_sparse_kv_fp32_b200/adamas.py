@@ -28,7 +28,7 @@ _lock = threading.Lock()
 _lib = None
 
 SYMBOLS = (
-    "adamas_status_string", "adamas_version", "adamas_workspace_bytes", "adamas_workspace_init",
+    "adamas_status_string", "adamas_version", "adamas_last_error_string", "adamas_workspace_bytes", "adamas_workspace_init",
     "adamas_encode_keys", "adamas_decode_step", "adamas_score", "adamas_get_device_error",
 )
 
@@ -36,7 +36,8 @@ SYMBOLS = (
 class AdamasError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where}: {status_string(status)} ({status})")
+        detail = f": {load().adamas_last_error_string().decode()}" if status == -4 else ""
+        super().__init__(f"{where}: {status_string(status)} ({status}){detail}")
 
 
 def load(path: str = LIBRARY) -> ctypes.CDLL:
@@ -53,6 +54,8 @@ def load(path: str = LIBRARY) -> ctypes.CDLL:
         l.adamas_status_string.restype = ctypes.c_char_p
         l.adamas_version.argtypes = []
         l.adamas_version.restype = I
+        l.adamas_last_error_string.argtypes = []
+        l.adamas_last_error_string.restype = ctypes.c_char_p
         l.adamas_workspace_bytes.argtypes = [I, I, I, I64, I, I]
         l.adamas_workspace_bytes.restype = SZ
         l.adamas_workspace_init.argtypes = [P, SZ, P]

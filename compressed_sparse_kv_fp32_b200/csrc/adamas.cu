@@ -116,18 +116,30 @@ struct DeviceInfo {
 
 static std::mutex g_mutex;
 static DeviceInfo g_devices[64];
+static thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+
+// Record a failed CUDA call for adamas_last_error_string and map it to a status.
+static int cuda_fail(cudaError_t e) {
+  g_last_cuda_error = e;
+  return ADAMAS_ERR_CUDA;
+}
+
+// Shared memory a block can use beyond the kernels' static shared memory.
+constexpr size_t kStaticSmemReserve = 1024;
 
 static int device_info(DeviceInfo** out) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ADAMAS_ERR_CUDA;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 0 || dev >= 64) return ADAMAS_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_mutex);
   DeviceInfo& d = g_devices[dev];
   if (d.sms == 0) {
     int sms = 0, optin = 0;
-    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
-      return ADAMAS_ERR_CUDA;
-    d.smem_optin = (size_t)optin;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess)
+      return cuda_fail(e);
+    d.smem_optin = (size_t)optin > kStaticSmemReserve ? (size_t)optin - kStaticSmemReserve : 0;
     d.sms = sms;
   }
   *out = &d;
@@ -181,9 +193,9 @@ static int launch_decode(const DecodeParams& prm, const WsLayout& L, DeviceInfo&
   {
     std::lock_guard<std::mutex> lock(g_mutex);
     if (!dev.attrs_set[G]) {
-      if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dev.smem_optin) !=
-          cudaSuccess)
-        return ADAMAS_ERR_CUDA;
+      const cudaError_t e =
+          cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dev.smem_optin);
+      if (e != cudaSuccess) return cuda_fail(e);
       dev.attrs_set[G] = true;
     }
   }
@@ -197,7 +209,8 @@ static int launch_decode(const DecodeParams& prm, const WsLayout& L, DeviceInfo&
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kernel, prm) != cudaSuccess) return ADAMAS_ERR_CUDA;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, prm);
+  if (e != cudaSuccess) return cuda_fail(e);
   return ADAMAS_OK;
 }
 
@@ -227,6 +240,10 @@ const char* adamas_status_string(int status) {
 
 int adamas_version(void) { return 100; }
 
+const char* adamas_last_error_string(void) {
+  return g_last_cuda_error == cudaSuccess ? "no CUDA error" : cudaGetErrorString(g_last_cuda_error);
+}
+
 size_t adamas_workspace_bytes(int B, int Hq, int Hkv, int64_t Nmax, int d, int budget) {
   if (check_shape(B, Hq, Hkv, Nmax, d, budget) != ADAMAS_OK) return 0;
   DeviceInfo* dev = nullptr;
@@ -238,7 +255,8 @@ size_t adamas_workspace_bytes(int B, int Hq, int Hkv, int64_t Nmax, int d, int b
 
 int adamas_workspace_init(void* workspace, size_t workspace_bytes, adamas_stream_t stream) {
   if (!workspace || workspace_bytes == 0) return ADAMAS_ERR_INVALID_ARG;
-  if (cudaMemsetAsync(workspace, 0, workspace_bytes, (cudaStream_t)stream) != cudaSuccess) return ADAMAS_ERR_CUDA;
+  const cudaError_t e = cudaMemsetAsync(workspace, 0, workspace_bytes, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e);
   return ADAMAS_OK;
 }
 
@@ -253,7 +271,8 @@ int adamas_encode_keys(const void* K, uint8_t* codes, const int32_t* pos_begin, 
   const dim3 grid((unsigned)((count + kEncThreads - 1) / kEncThreads), (unsigned)(B * Hkv));
   encode_keys_kernel<<<grid, kEncThreads, 0, (cudaStream_t)stream>>>(
       static_cast<const uint16_t*>(K), codes, pos_begin, count, Hkv, Nmax);
-  if (cudaGetLastError() != cudaSuccess) return ADAMAS_ERR_CUDA;
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e);
   return ADAMAS_OK;
 }
 
@@ -309,7 +328,10 @@ int adamas_decode_step(const void* q, const uint8_t* codes, const void* K, const
     case 8: rc = launch_decode<8>(prm, L, *dev, st); break;
     default: rc = ADAMAS_ERR_UNSUPPORTED;
   }
-  if (rc == ADAMAS_OK && cudaGetLastError() != cudaSuccess) rc = ADAMAS_ERR_CUDA;
+  if (rc == ADAMAS_OK) {
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) rc = cuda_fail(e);
+  }
   return rc;
 }
 
@@ -336,7 +358,8 @@ int adamas_score(const void* q, const uint8_t* codes, const int32_t* seq_lens, i
     case 8: launch_score<8>(grid, st, qq, codes, seq_lens, Hq, Hkv, Nmax, dist); break;
     default: return ADAMAS_ERR_UNSUPPORTED;
   }
-  if (cudaGetLastError() != cudaSuccess) return ADAMAS_ERR_CUDA;
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e);
   return ADAMAS_OK;
 }
 
@@ -345,10 +368,10 @@ int adamas_get_device_error(const void* workspace, size_t workspace_bytes, uint3
   if (!workspace || !error_word || workspace_bytes < 64 * sizeof(uint32_t)) return ADAMAS_ERR_INVALID_ARG;
   uint32_t word = 0;
   cudaStream_t st = (cudaStream_t)stream;
-  if (cudaMemcpyAsync(&word, static_cast<const uint32_t*>(workspace) + 2, sizeof word, cudaMemcpyDeviceToHost, st) !=
-          cudaSuccess ||
-      cudaStreamSynchronize(st) != cudaSuccess)
-    return ADAMAS_ERR_CUDA;
+  cudaError_t e = cudaMemcpyAsync(&word, static_cast<const uint32_t*>(workspace) + 2, sizeof word,
+                                  cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e);
   *error_word = word;
   return word == 0 ? ADAMAS_OK : ADAMAS_ERR_DEVICE;
 }

@@ -417,12 +417,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const DecodePa
     for (int e = 0; e < 8; ++e) o[e] = 0.0f;
 
     const int32_t* idx_h = p.idx + hq * p.budget + j0;
-    for (int64_t j = hw; j < slen; j += 2 * kWarps * kRowsPerHalfWarp) {
+    // The trip count depends on the warp only, so both half-warps always reach
+    // the full-warp shuffles below together.
+    for (int64_t jb = 2 * warp; jb < slen; jb += 2 * kWarps * kRowsPerHalfWarp) {
       int32_t t[kRowsPerHalfWarp];
       uint4 kr[kRowsPerHalfWarp], vr[kRowsPerHalfWarp];
 #pragma unroll
       for (int u2 = 0; u2 < kRowsPerHalfWarp; ++u2) {
-        const int64_t jj = j + (int64_t)u2 * 2 * kWarps;
+        const int64_t jj = jb + (hw & 1) + (int64_t)u2 * 2 * kWarps;
         t[u2] = jj < slen ? __ldcg(idx_h + jj) : -1;
         if (t[u2] >= len_b) t[u2] = -1;  // never read outside the sequence
       }

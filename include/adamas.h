@@ -71,6 +71,10 @@ const char *adamas_status_string(int status);
 /* Library version, major * 10000 + minor * 100 + patch. */
 int adamas_version(void);
 
+/* Text of the last CUDA error that made a call of this thread return
+ * ADAMAS_ERR_CUDA ("no CUDA error" if none).  Never NULL. */
+const char *adamas_last_error_string(void);
+
 /*
  * Bytes of device workspace adamas_decode_step needs for these sizes on the
  * current CUDA device (0 when the sizes are unsupported).  The workspace holds
