@@ -30,6 +30,7 @@ _lib = None
 SYMBOLS = (
     "adamas_status_string", "adamas_version", "adamas_last_error_string", "adamas_workspace_bytes", "adamas_workspace_init",
     "adamas_encode_keys", "adamas_decode_step", "adamas_score", "adamas_get_device_error",
+    "adamas_decode_step_static",
 )
 
 
@@ -68,6 +69,8 @@ def load(path: str = LIBRARY) -> ctypes.CDLL:
         l.adamas_score.restype = I
         l.adamas_get_device_error.argtypes = [P, SZ, ctypes.POINTER(ctypes.c_uint32), P]
         l.adamas_get_device_error.restype = I
+        l.adamas_decode_step_static.argtypes = [P, P, P, P, P, I, I, I, I64, I, I, P, P, P]
+        l.adamas_decode_step_static.restype = I
         _lib = l
         return l
 

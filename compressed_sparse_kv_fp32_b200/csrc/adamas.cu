@@ -377,3 +377,107 @@ int adamas_get_device_error(const void* workspace, size_t workspace_bytes, uint3
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------ decode step without a caller workspace
+// Some callers cannot allocate device memory at the point where they decode: a
+// custom allocator that must not be re-entered from inside a serving loop, a
+// framework hook that runs with allocation forbidden, or a host program that only
+// ever receives pointers to memory someone else owns.  adamas_decode_step_static
+// serves them: it uses a fixed scratch array that the library itself holds in
+// every device's global memory (a file-scope __device__ array, reserved when the
+// library's module is loaded onto a device and kept until the process exits),
+// so it needs no workspace argument and calls no allocator.
+namespace adamas {
+
+constexpr size_t kStaticScratchBytes = size_t(4) << 20;  // 4 MiB on every device that loads the library
+
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+static std::mutex g_static_mutex;
+static void* g_static_scratch_ptr[64] = {};
+
+// Device address of g_static_scratch on the current device.  In host code the
+// array's name is only a host-side stand-in, so the address is looked up once
+// per device, with that device current, and cached.
+static int static_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 0 || dev >= 64) return ADAMAS_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_static_mutex);
+  if (!g_static_scratch_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess) return cuda_fail(e);
+    g_static_scratch_ptr[dev] = p;
+  }
+  *out = g_static_scratch_ptr[dev];
+  return ADAMAS_OK;
+}
+
+}  // namespace adamas
+
+extern "C" int adamas_decode_step_static(const void* q, const uint8_t* codes, const void* K, const void* V,
+                                         const int32_t* seq_lens, int B, int Hq, int Hkv, int64_t Nmax, int d,
+                                         int budget, float* out, int32_t* idx, adamas_stream_t stream) {
+  int rc = check_shape(B, Hq, Hkv, Nmax, d, budget);
+  if (rc != ADAMAS_OK) return rc;
+  if (B == 0) return ADAMAS_OK;
+  if (!q || !seq_lens || !out || (budget > 0 && !idx)) return ADAMAS_ERR_INVALID_ARG;
+  if (Nmax > 0 && (!codes || !K || !V)) return ADAMAS_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(codes, 32) || !aligned(K, 16) || !aligned(V, 16) || !aligned(out, 16) ||
+      !aligned(idx, 4) || !aligned(seq_lens, 4))
+    return ADAMAS_ERR_INVALID_ARG;
+  DeviceInfo* dev = nullptr;
+  if ((rc = device_info(&dev)) != ADAMAS_OK) return rc;
+  WsLayout L;
+  if ((rc = ws_layout(B, Hq, Hkv, Nmax, budget, *dev, &L)) != ADAMAS_OK) return rc;
+  if (L.total > kStaticScratchBytes) return ADAMAS_ERR_WORKSPACE;  // sizes beyond the fixed scratch
+  void* scratch = nullptr;
+  if ((rc = static_scratch(&scratch)) != ADAMAS_OK) return rc;
+
+  // The scratch keeps whatever the previous call left; the grid-wait counters,
+  // the error word and the per-head tickets must start at zero.
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e = cudaMemsetAsync(scratch, 0, L.hist, st);
+  if (e != cudaSuccess) return cuda_fail(e);
+
+  unsigned char* ws = static_cast<unsigned char*>(scratch);
+  DecodeParams prm;
+  prm.q = static_cast<const uint16_t*>(q);
+  prm.codes = codes;
+  prm.K = static_cast<const uint16_t*>(K);
+  prm.V = static_cast<const uint16_t*>(V);
+  prm.seq_lens = seq_lens;
+  prm.out = out;
+  prm.idx = idx;
+  prm.ctrl = reinterpret_cast<uint32_t*>(ws + L.ctrl);
+  prm.head_done = reinterpret_cast<uint32_t*>(ws + L.head_done);
+  prm.hist = reinterpret_cast<uint32_t*>(ws + L.hist);
+  prm.partial = reinterpret_cast<float*>(ws + L.partial);
+  prm.dglobal = L.smem_d ? nullptr : reinterpret_cast<uint16_t*>(ws + L.dspill);
+  prm.B = B;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.Nmax = Nmax;
+  prm.budget = budget;
+  prm.S = L.S;
+  prm.range_cap = L.range_cap;
+  prm.smem_d = L.smem_d ? 1 : 0;
+  switch (Hq / Hkv) {
+    case 1: rc = launch_decode<1>(prm, L, *dev, st); break;
+    case 2: rc = launch_decode<2>(prm, L, *dev, st); break;
+    case 3: rc = launch_decode<3>(prm, L, *dev, st); break;
+    case 4: rc = launch_decode<4>(prm, L, *dev, st); break;
+    case 5: rc = launch_decode<5>(prm, L, *dev, st); break;
+    case 6: rc = launch_decode<6>(prm, L, *dev, st); break;
+    case 7: rc = launch_decode<7>(prm, L, *dev, st); break;
+    case 8: rc = launch_decode<8>(prm, L, *dev, st); break;
+    default: rc = ADAMAS_ERR_UNSUPPORTED;
+  }
+  if (rc == ADAMAS_OK) {
+    e = cudaGetLastError();
+    if (e != cudaSuccess) rc = cuda_fail(e);
+  }
+  return rc;
+}

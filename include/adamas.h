@@ -137,6 +137,33 @@ int adamas_score(const void *q, const uint8_t *codes, const int32_t *seq_lens, i
                  int Hkv, int64_t Nmax, int d, uint16_t *dist, adamas_stream_t stream);
 
 /*
+ * adamas_decode_step for callers that cannot allocate device memory where they
+ * decode -- an allocator that must not be re-entered from the decode loop, a hook
+ * that runs with allocation forbidden, or a program that only receives pointers
+ * to memory someone else owns.  The ADAMAS article has no counterpart of this
+ * entry point; it is a property of this library.
+ *
+ * Same arguments, results and rules as adamas_decode_step, without the
+ * workspace: the scratch is a fixed 4 MiB array that the library keeps in the
+ * global memory of every device it is loaded on, until the process exits.
+ * Nothing is allocated or freed by this call.
+ *   - Sizes whose workspace (adamas_workspace_bytes) exceeds 4 MiB are rejected
+ *     with ADAMAS_ERR_WORKSPACE before anything is enqueued; use
+ *     adamas_decode_step for those.
+ *   - The first call on each device looks up the array's device address (a
+ *     one-time set-up); make that first call before any stream capture.
+ *   - Every call on a device shares the one array, and it keeps the previous
+ *     call's contents.  The call clears what must start at zero, but calls that
+ *     may overlap on the GPU (different streams, or different threads without
+ *     ordering) race on it; serialise them.
+ *   - The device error word lives in the shared array and is cleared by the next
+ *     call; it cannot be read back through this entry point.
+ */
+int adamas_decode_step_static(const void *q, const uint8_t *codes, const void *K, const void *V,
+                              const int32_t *seq_lens, int B, int Hq, int Hkv, int64_t Nmax, int d,
+                              int budget, float *out, int32_t *idx, adamas_stream_t stream);
+
+/*
  * Synchronise `stream`, then copy the workspace's device error word into
  * *error_word (ADAMAS_DEVERR_* bits).  Returns ADAMAS_OK when the word is zero,
  * ADAMAS_ERR_DEVICE when it is not.
