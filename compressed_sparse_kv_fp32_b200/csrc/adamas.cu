@@ -125,7 +125,7 @@ static int cuda_fail(cudaError_t e) {
 }
 
 // Shared memory a block can use beyond the kernels' static shared memory.
-constexpr size_t kStaticSmemReserve = 1024;
+constexpr size_t kStaticSmemReserve = 8192;
 
 static int device_info(DeviceInfo** out) {
   int dev = 0;
@@ -151,6 +151,8 @@ struct WsLayout {
   int S;
   int64_t range_cap;
   bool smem_d;
+  int nstages;
+  int row_cap;
   size_t smem;
 };
 
@@ -170,17 +172,31 @@ static int ws_layout(int B, int Hq, int Hkv, int64_t Nmax, int budget, const Dev
   const int G = Hq / Hkv;
   const int64_t umax = (int64_t)B * Hkv * Nmax;
   int64_t want = (umax + 2047) / 2048;
-  L->S = (int)(want < 1 ? 1 : (want > dev.sms ? dev.sms : want));
+  const int max_blocks = dev.sms < kMaxBlocks ? dev.sms : kMaxBlocks;
+  L->S = (int)(want < 1 ? 1 : (want > max_blocks ? max_blocks : want));
   L->range_cap = umax > 0 ? (umax + L->S - 1) / L->S : 1;
-  L->smem_d = DecodeSmem::total(B, G, L->range_cap, true) <= dev.smem_optin;
-  L->smem = DecodeSmem::total(B, G, L->range_cap, L->smem_d);
+  if (L->range_cap >= (int64_t(1) << 23)) return ADAMAS_ERR_UNSUPPORTED;  // token offsets are packed in 23 bits
+  // Distances in shared memory with the deepest ring that still fits; else the
+  // distances go to the workspace and the ring keeps all its stages.
+  L->smem_d = false;
+  L->nstages = kStages;
+  for (int st = kStages; st >= kMinStages; --st) {
+    if (DecodeSmem::total(B, G, L->range_cap, true, st) <= dev.smem_optin) {
+      L->smem_d = true;
+      L->nstages = st;
+      break;
+    }
+  }
+  L->smem = DecodeSmem::total(B, G, L->range_cap, L->smem_d, L->nstages);
+  L->row_cap = DecodeSmem::row_cap(G, L->range_cap, L->smem_d, L->nstages);
   if (L->smem > dev.smem_optin) return ADAMAS_ERR_UNSUPPORTED;
   size_t off = 0;
   L->ctrl = off;      off += align256(64 * sizeof(uint32_t));
   L->head_done = off; off += align256((size_t)B * Hq * sizeof(uint32_t));
   L->hist = off;      off += align256((size_t)(L->S + B * Hkv) * G * kHistStride * sizeof(uint32_t));
   L->partial = off;   off += align256((size_t)(L->S + B * Hq) * kPartial * sizeof(float));
-  L->dspill = off;    off += L->smem_d ? 0 : align256((size_t)L->S * G * L->range_cap * sizeof(uint16_t));
+  L->dspill = off;
+  off += L->smem_d ? 0 : align256((size_t)L->S * G * DecodeSmem::dstride(L->range_cap) * sizeof(uint16_t));
   L->total = off;
   return ADAMAS_OK;
 }
@@ -315,6 +331,8 @@ int adamas_decode_step(const void* q, const uint8_t* codes, const void* K, const
   prm.S = L.S;
   prm.range_cap = L.range_cap;
   prm.smem_d = L.smem_d ? 1 : 0;
+  prm.row_cap = L.row_cap;
+  prm.nstages = L.nstages;
 
   cudaStream_t st = (cudaStream_t)stream;
   switch (Hq / Hkv) {
@@ -464,6 +482,8 @@ extern "C" int adamas_decode_step_static(const void* q, const uint8_t* codes, co
   prm.S = L.S;
   prm.range_cap = L.range_cap;
   prm.smem_d = L.smem_d ? 1 : 0;
+  prm.row_cap = L.row_cap;
+  prm.nstages = L.nstages;
   switch (Hq / Hkv) {
     case 1: rc = launch_decode<1>(prm, L, *dev, st); break;
     case 2: rc = launch_decode<2>(prm, L, *dev, st); break;
