@@ -111,7 +111,7 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(const uint16_t* __
 struct DeviceInfo {
   int sms = 0;
   size_t smem_optin = 0;
-  bool attrs_set[kMaxGroup + 1] = {};
+  bool attrs_set[2][kMaxGroup + 1] = {};
 };
 
 static std::mutex g_mutex;
@@ -151,7 +151,6 @@ struct WsLayout {
   int S;
   int64_t range_cap;
   bool smem_d;
-  int nstages;
   int row_cap;
   size_t smem;
 };
@@ -175,26 +174,32 @@ static int ws_layout(int B, int Hq, int Hkv, int64_t Nmax, int budget, const Dev
   const int max_blocks = dev.sms < kMaxBlocks ? dev.sms : kMaxBlocks;
   L->S = (int)(want < 1 ? 1 : (want > max_blocks ? max_blocks : want));
   L->range_cap = umax > 0 ? (umax + L->S - 1) / L->S : 1;
-  if (L->range_cap >= (int64_t(1) << 23)) return ADAMAS_ERR_UNSUPPORTED;  // token offsets are packed in 23 bits
-  // Distances in shared memory with the deepest ring that still fits; else the
-  // distances go to the workspace and the ring keeps all its stages.
-  L->smem_d = false;
-  L->nstages = kStages;
-  for (int st = kStages; st >= kMinStages; --st) {
-    if (DecodeSmem::total(B, G, L->range_cap, true, st) <= dev.smem_optin) {
-      L->smem_d = true;
-      L->nstages = st;
-      break;
-    }
+  // With equal lengths the kernel may split over a multiple of the kv-head count
+  // (each block within one head): its shares are at most ceil(Nmax / (S / heads)).
+  const int64_t heads = (int64_t)B * Hkv;
+  if (heads > 0 && heads <= L->S) {
+    const int64_t per_head = L->S / heads;
+    const int64_t r2 = (Nmax + per_head - 1) / per_head;
+    if (r2 > L->range_cap) L->range_cap = r2;
   }
-  L->smem = DecodeSmem::total(B, G, L->range_cap, L->smem_d, L->nstages);
-  L->row_cap = DecodeSmem::row_cap(G, L->range_cap, L->smem_d, L->nstages);
+  if (L->range_cap >= (int64_t(1) << 23)) return ADAMAS_ERR_UNSUPPORTED;  // token offsets are packed in 23 bits
+  // Distances in shared memory when they fit beside the smallest gather staging;
+  // the staging then takes what is left (an even number of rows).
+  const size_t fixed = DecodeSmem::fixed(B, G);
+  const size_t dist = DecodeSmem::align128(DecodeSmem::dist(G, L->range_cap, true));
+  L->smem_d = fixed + dist + (size_t)kMinRowsStaged * kRowBytes <= dev.smem_optin;
+  const size_t left = dev.smem_optin - fixed - (L->smem_d ? dist : 0);
+  if (dev.smem_optin < fixed + (size_t)kMinRowsStaged * kRowBytes) return ADAMAS_ERR_UNSUPPORTED;
+  size_t rows = left / kRowBytes;
+  if (rows > (size_t)kMaxRowsStaged) rows = kMaxRowsStaged;
+  L->row_cap = (int)(rows & ~(size_t)1);
+  L->smem = DecodeSmem::total(B, G, L->range_cap, L->smem_d, L->row_cap);
   if (L->smem > dev.smem_optin) return ADAMAS_ERR_UNSUPPORTED;
   size_t off = 0;
   L->ctrl = off;      off += align256(64 * sizeof(uint32_t));
   L->head_done = off; off += align256((size_t)B * Hq * sizeof(uint32_t));
   L->hist = off;      off += align256((size_t)(L->S + B * Hkv) * G * kHistStride * sizeof(uint32_t));
-  L->partial = off;   off += align256((size_t)(L->S + B * Hq) * kPartial * sizeof(float));
+  L->partial = off;   off += align256((size_t)(L->S + B * Hkv) * G * kPartial * sizeof(float));
   L->dspill = off;
   off += L->smem_d ? 0 : align256((size_t)L->S * G * DecodeSmem::dstride(L->range_cap) * sizeof(uint16_t));
   L->total = off;
@@ -205,14 +210,14 @@ static bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
 
 template <int G>
 static int launch_decode(const DecodeParams& prm, const WsLayout& L, DeviceInfo& dev, cudaStream_t stream) {
-  auto kernel = decode_step_kernel<G>;
+  auto kernel = prm.smem_d ? decode_step_kernel<G, true> : decode_step_kernel<G, false>;
   {
     std::lock_guard<std::mutex> lock(g_mutex);
-    if (!dev.attrs_set[G]) {
+    if (!dev.attrs_set[prm.smem_d ? 1 : 0][G]) {
       const cudaError_t e =
           cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dev.smem_optin);
       if (e != cudaSuccess) return cuda_fail(e);
-      dev.attrs_set[G] = true;
+      dev.attrs_set[prm.smem_d ? 1 : 0][G] = true;
     }
   }
   cudaLaunchConfig_t cfg = {};
@@ -332,7 +337,6 @@ int adamas_decode_step(const void* q, const uint8_t* codes, const void* K, const
   prm.range_cap = L.range_cap;
   prm.smem_d = L.smem_d ? 1 : 0;
   prm.row_cap = L.row_cap;
-  prm.nstages = L.nstages;
 
   cudaStream_t st = (cudaStream_t)stream;
   switch (Hq / Hkv) {
@@ -483,7 +487,6 @@ extern "C" int adamas_decode_step_static(const void* q, const uint8_t* codes, co
   prm.range_cap = L.range_cap;
   prm.smem_d = L.smem_d ? 1 : 0;
   prm.row_cap = L.row_cap;
-  prm.nstages = L.nstages;
   switch (Hq / Hkv) {
     case 1: rc = launch_decode<1>(prm, L, *dev, st); break;
     case 2: rc = launch_decode<2>(prm, L, *dev, st); break;

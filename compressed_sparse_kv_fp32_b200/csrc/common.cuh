@@ -16,6 +16,7 @@ constexpr int kMaxBatch = 1024;
 // Bits of the device error word (mirrors ADAMAS_DEVERR_* in adamas.h).
 constexpr uint32_t kErrSeqLen = 0x1u;
 constexpr uint32_t kErrTimeout = 0x2u;
+constexpr uint32_t kErrInternal = 0x4u;
 
 // RN_fp32(1/sqrt(128)), bit pattern 0x3DB504F3: the rotation's normalisation.
 __device__ __forceinline__ float hadamard_norm() { return __uint_as_float(0x3DB504F3u); }
@@ -98,8 +99,10 @@ __device__ __forceinline__ void red_add_release_gpu64(unsigned long long* p, uns
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)), "l"(src) : "memory");
 }
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 // Bring the 128-byte line holding `p` into L2, to be kept there preferentially.

@@ -8,37 +8,36 @@
 // vectors).
 //
 // Work split.  All (b, kv head, token) units of the batch form one range that is
-// cut evenly over the S blocks; a block's share may cross kv heads, so it is
-// handled as "segments" (the part of one kv head inside the block's share).
-//   phase 1  per segment: encode the G query heads of the kv head; stream the
-//            segment's packed codes through a ring of 32 KiB shared-memory
-//            stages filled by bulk asynchronous copies (cp.async.bulk, one
-//            mbarrier per stage, all but one stage in flight); each thread scores
-//            two code rows per stage (G distances each), keeps the distances in
-//            shared memory and adds them to one 385-bin histogram per query
-//            head; the histograms are published to the workspace.
+// cut evenly over Sr <= S blocks (when every sequence has the same length and
+// there are no more kv heads than blocks, Sr is a multiple of the number of kv
+// heads so that no block straddles two heads); a block's share is handled as
+// "segments" (the part of one kv head inside the block's share).
+//   phase 1  per segment: encode the G query heads of the kv head, stream the
+//            packed code rows with 32-byte loads (each thread keeps the next rows
+//            in flight while it scores the current ones), keep the G distances of
+//            every token in shared memory and add them to one 385-bin histogram
+//            per query head; publish the histograms.
 //   -- grid-wide wait --
 //   phase 2  per segment and query head: sum the head's histograms (one per
 //            segment of that head, loaded together) to get the threshold T with
-//            count(D < T) < k_eff <= count(D <= T).  Each warp scans its slice of
-//            the distances eight at a time and compacts the tokens with D <= T,
-//            in index order, into a list; then every listed token goes straight
-//            to its final slot of the (D, index)-ordered output:
-//            slot = #tokens with smaller D + #tokens with equal D and a lower
-//            index (earlier segments from their histograms, earlier warps from
-//            per-warp counts, earlier lanes by a warp match).  Slots >= k_eff are
-//            dropped, which keeps ties at T for the lowest indices.  The K and V
-//            rows of every kept token are prefetched into L2 on the spot.
-//   -- grid-wide wait --
-//   phase 3  the kept rows of all query heads form a second range, cut evenly
-//            over the blocks; each block stages its rows' K and V in shared
-//            memory with 16-byte cp.async copies, every half-warp keeps an
-//            online-softmax state over its rows, the block publishes one partial
-//            state per query head it touched, and the last block to finish a
-//            query head (atomic ticket, no waiting) merges the partials into out.
+//            count(D < T) < k_eff <= count(D <= T).  Pass 1: each warp scans its
+//            slice of the distances eight at a time and counts the tokens with
+//            D <= T per distance; prefix sums over warps then give every warp
+//            the number of tokens it keeps and where its kept tokens go in a
+//            block list.  Pass 2: each warp scans again in index order and puts
+//            every candidate straight at its final slot of the (D, index)-ordered
+//            output: slot = #tokens with smaller D + #tokens with equal D and a
+//            lower index (earlier segments from their histograms, earlier warps
+//            from the per-warp counts, earlier lanes by a warp match).  Slots
+//            >= k_eff are dropped, which keeps ties at T for the lowest indices.
+//            The block then gathers the K and V rows of its kept tokens (16-byte
+//            cp.async copies, double-buffered), every half-warp keeps an
+//            online-softmax state, and the block publishes one partial state for
+//            the query head; the last block to publish for a query head (atomic
+//            ticket, no waiting) merges the partials into out.
 //
-// Every wait is bounded: a grid-wide wait gives up after kSpinLimit polls and a
-// stage wait after kMbarLimit polls; either sets ADAMAS_DEVERR_TIMEOUT.
+// The grid-wide wait is bounded: it gives up after kSpinLimit polls and sets
+// ADAMAS_DEVERR_TIMEOUT.
 #pragma once
 
 #include "common.cuh"
@@ -51,16 +50,13 @@ constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
 constexpr int kHistStride = 388;                     // >= kBins, multiple of 4
 constexpr int kPartial = 132;                        // m, l, pad, pad, o[128]
-constexpr int kRowsPerThread = 2;                    // code rows per thread per stage
-constexpr int kStageTokens = kThreads * kRowsPerThread;
-constexpr uint32_t kStageBytes = kStageTokens * kCodeBytes;  // 32 KiB
-constexpr int kStages = 4;                           // most ring stages (fewer when shared memory is short)
-constexpr int kMinStages = 2;
 constexpr uint32_t kRowBytes = 2 * kDim * 2;         // one K row + one V row (bf16)
-constexpr int kMaxRowsStaged = 512;
+constexpr int kScratch = 256;                        // candidate entries per warp per 256-token group
+constexpr int kMaxKept = 2048;                       // kept tokens listed per sweep
+constexpr int kMaxRowsStaged = 256;
+constexpr int kMinRowsStaged = 32;
 constexpr int kMaxBlocks = 1024;
 constexpr uint32_t kSpinLimit = 1u << 20;            // grid-wide wait polls (about a second)
-constexpr uint32_t kMbarLimit = 1u << 20;            // stage wait polls
 
 struct DecodeParams {
   const uint16_t* q;
@@ -71,9 +67,9 @@ struct DecodeParams {
   float* out;
   int32_t* idx;
   uint32_t* ctrl;       // [0..1] grid-wait word (generation << 32 | arrivals), [2] error word
-  uint32_t* head_done;  // [B*Hq] tickets of phase 3
+  uint32_t* head_done;  // [B*Hq] merge tickets
   uint32_t* hist;       // [(S + B*Hkv) * G][kHistStride]
-  float* partial;       // [(S + B*Hq)][kPartial]
+  float* partial;       // [(S + B*Hkv) * G][kPartial]
   uint16_t* dglobal;    // [S][G][dstride] when distances do not fit in shared memory
   int B, Hq, Hkv;
   int64_t Nmax;
@@ -81,37 +77,31 @@ struct DecodeParams {
   int S;
   int64_t range_cap;    // >= units of any block
   int smem_d;           // distances kept in shared memory
-  int row_cap;          // K/V rows staged per chunk in phase 3
-  int nstages;          // ring stages in phase 1, kMinStages..kStages
+  int row_cap;          // K/V rows staged per gather buffer pair (even)
 };
 
 // Shared-memory carve-up (bytes), shared with the host.
 struct DecodeSmem {
   static __host__ __device__ inline size_t align128(size_t x) { return (x + 127) / 128 * 128; }
-  static __host__ __device__ inline size_t meta(int B) { return (size_t)(B + 1) * 16 + (size_t)B * 4; }
+  static __host__ __device__ inline size_t meta(int B) { return (size_t)(B + 1) * 8 + (size_t)B * 4; }
   static __host__ __device__ inline size_t qwords(int G) { return (size_t)G * kCodeWords * 4; }
-  // histograms (phase 1), per-warp counts + rank bases + round totals (phase 2),
-  // half-warp softmax states (phase 3)
+  // histograms (phase 1); per-warp counts + rank bases, then the half-warp
+  // softmax states (phase 2)
   static __host__ __device__ inline size_t work(int G) {
-    const int rows = G > kWarps + 2 ? G : kWarps + 2;
+    const int rows = G > kWarps + 1 ? G : kWarps + 1;
     return (size_t)rows * kHistStride * 4;
   }
-  static __host__ __device__ inline size_t rowidx() { return (size_t)kMaxRowsStaged * 4; }
-  static __host__ __device__ inline size_t ring(int nstages) { return (size_t)nstages * kStageBytes; }
+  static __host__ __device__ inline size_t scratch() { return (size_t)kWarps * kScratch * 4; }
+  static __host__ __device__ inline size_t kept() { return (size_t)kMaxKept * 4; }
   static __host__ __device__ inline int64_t dstride(int64_t range_cap) { return (range_cap + 63) / 64 * 64; }
   static __host__ __device__ inline size_t dist(int G, int64_t range_cap, bool in_smem) {
     return in_smem ? (size_t)G * (size_t)dstride(range_cap) * 2 : 0;
   }
-  static __host__ __device__ inline size_t big(int G, int64_t range_cap, bool in_smem, int nstages) {
-    return ring(nstages) + dist(G, range_cap, in_smem);
+  static __host__ __device__ inline size_t fixed(int B, int G) {
+    return align128(meta(B)) + align128(qwords(G)) + align128(work(G)) + align128(scratch()) + align128(kept());
   }
-  static __host__ __device__ inline size_t total(int B, int G, int64_t range_cap, bool in_smem, int nstages) {
-    return align128(meta(B)) + align128(qwords(G)) + align128(work(G)) + align128(rowidx()) +
-           align128(big(G, range_cap, in_smem, nstages));
-  }
-  static __host__ __device__ inline int row_cap(int G, int64_t range_cap, bool in_smem, int nstages) {
-    const size_t rows = big(G, range_cap, in_smem, nstages) / kRowBytes;
-    return (int)(rows < (size_t)kMaxRowsStaged ? rows : (size_t)kMaxRowsStaged);
+  static __host__ __device__ inline size_t total(int B, int G, int64_t range_cap, bool in_smem, int row_cap) {
+    return fixed(B, G) + align128(dist(G, range_cap, in_smem)) + (size_t)row_cap * kRowBytes;
   }
 };
 
@@ -225,15 +215,63 @@ __device__ __forceinline__ Segment segment_at(int64_t u, int64_t lo, int64_t hi,
   return g;
 }
 
+// ------------------------------------------------------------------ phase-1 helpers
+// Rows base + j*kThreads + tid (j < U) of a segment's code rows, 32 bytes each.
+template <int U>
+__device__ __forceinline__ void load_rows(uint32_t (&dst)[U][kCodeWords], const uint8_t* crow, int base,
+                                          int seg_len, int tid) {
+#pragma unroll
+  for (int j = 0; j < U; ++j) {
+    const int t = base + j * kThreads + tid;
+    if (t < seg_len) ld_stream_v8(crow + (size_t)t * kCodeBytes, dst[j]);
+  }
+}
+
+// Distances of those rows to the G query codes: stored at dseg[g*dstride + t]
+// and counted in the per-head histograms.
+template <int G, int U>
+__device__ __forceinline__ void score_rows(const uint32_t (&src)[U][kCodeWords], const uint32_t (&qw)[G][kCodeWords],
+                                           int base, int seg_len, int tid, uint16_t* dseg, int64_t dstride,
+                                           uint32_t* hist) {
+#pragma unroll
+  for (int j = 0; j < U; ++j) {
+    const int t = base + j * kThreads + tid;
+    if (t < seg_len) {
+      uint32_t e[kCodeWords];
+      key_odd_mask(src[j], e);
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const int d = l1_distance(src[j], e, qw[g]);
+        dseg[(size_t)g * dstride + t] = (uint16_t)d;
+        atomicAdd(&hist[g * kHistStride + d], 1u);
+      }
+    }
+  }
+}
+
+// Distances of eight consecutive positions 8*grp .. 8*grp+7 (0xFFFF where grp is
+// past the warp's slice).
+__device__ __forceinline__ void load_dist8(const uint16_t* drow, int grp, bool in, uint32_t (&d)[8]) {
+  uint4 v = make_uint4(0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu);
+  if (in) v = *reinterpret_cast<const uint4*>(drow + (size_t)grp * 8);
+  d[0] = v.x & 0xFFFFu; d[1] = v.x >> 16; d[2] = v.y & 0xFFFFu; d[3] = v.y >> 16;
+  d[4] = v.z & 0xFFFFu; d[5] = v.z >> 16; d[6] = v.w & 0xFFFFu; d[7] = v.w >> 16;
+}
+
 // ------------------------------------------------------------------ the kernel
-template <int G>
+// SMEM_D: the distances of the block's share live in shared memory (else in the
+// workspace).
+template <int G, bool SMEM_D>
 __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const DecodeParams p) {
   extern __shared__ __align__(128) unsigned char smem[];
-  __shared__ uint64_t sm_full[kStages];
   __shared__ int sm_flag;
   __shared__ int sm_T;
   __shared__ int sm_last;
   __shared__ int sm_nlist;
+  __shared__ int sm_kept_total;
+  __shared__ int sm_wlt[kWarps];    // per warp: candidates with D < T
+  __shared__ int sm_weq[kWarps];    // per warp: candidates with D == T
+  __shared__ int sm_wkept[kWarps];  // per warp: first position of its kept tokens in the block list
   __shared__ int64_t sm_scan[kWarps + 1];
   __shared__ int sm_list[kMaxBlocks];
 
@@ -242,34 +280,35 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const DecodePa
   const uint32_t lt = (1u << lane) - 1u;
 
   int64_t* sm_uoff = reinterpret_cast<int64_t*>(smem);                  // [B + 1]
-  int64_t* sm_roff = sm_uoff + (B + 1);                                 // [B + 1]
-  int32_t* sm_len = reinterpret_cast<int32_t*>(sm_roff + (B + 1));      // [B]
+  int32_t* sm_len = reinterpret_cast<int32_t*>(sm_uoff + (B + 1));      // [B]
   unsigned char* cur = smem + DecodeSmem::align128(DecodeSmem::meta(B));
   uint32_t* sm_q = reinterpret_cast<uint32_t*>(cur);                    // [G][8]
   cur += DecodeSmem::align128(DecodeSmem::qwords(G));
   uint32_t* sm_work = reinterpret_cast<uint32_t*>(cur);                 // [rows][kHistStride]
   cur += DecodeSmem::align128(DecodeSmem::work(G));
-  int32_t* sm_rowidx = reinterpret_cast<int32_t*>(cur);                 // [kMaxRowsStaged]
-  cur += DecodeSmem::align128(DecodeSmem::rowidx());
-  unsigned char* sm_big = cur;  // phase 1: ring | distances; phase 2: candidate lists | distances; phase 3: rows
-
-  const int nstages = p.nstages;
+  uint32_t* sm_scratch = reinterpret_cast<uint32_t*>(cur);              // [kWarps][kScratch]
+  cur += DecodeSmem::align128(DecodeSmem::scratch());
+  int32_t* sm_kept = reinterpret_cast<int32_t*>(cur);                   // [kMaxKept]
+  cur += DecodeSmem::align128(DecodeSmem::kept());
   const int64_t dstride = DecodeSmem::dstride(p.range_cap);
-  uint16_t* dbuf = p.smem_d ? reinterpret_cast<uint16_t*>(sm_big + DecodeSmem::ring(nstages))
-                            : p.dglobal + (int64_t)s * G * dstride;
+  uint16_t* dbuf;
+  if constexpr (SMEM_D) {
+    dbuf = reinterpret_cast<uint16_t*>(cur);                            // [G][dstride]
+    cur += DecodeSmem::align128(DecodeSmem::dist(G, p.range_cap, true));
+  } else {
+    dbuf = p.dglobal + (int64_t)s * G * dstride;
+  }
+  unsigned char* sm_rows = cur;                                         // [row_cap][512]
 
   uint32_t gen0 = 0;
-  if (tid == 0) {
-    for (int k = 0; k < nstages; ++k) mbar_init(&sm_full[k], 1);
-    fence_mbar_init();
-    gen0 = (uint32_t)(ld_relaxed_gpu64(reinterpret_cast<const unsigned long long*>(p.ctrl)) >> 32);
-  }
+  if (tid == 0) gen0 = (uint32_t)(ld_relaxed_gpu64(reinterpret_cast<const unsigned long long*>(p.ctrl)) >> 32);
 
-  // ---- lengths and offsets of the unit range and of the kept-row range
-  int64_t uoff_total, roff_total;
+  // ---- lengths and unit offsets per sequence
+  int64_t U;
+  int uniform;
   {
     // B <= kMaxBatch = 2 * kThreads: thread i owns batches 2i and 2i+1
-    int64_t lu = 0, lr = 0;
+    int64_t lu = 0;
     for (int k = 0; k < 2; ++k) {
       const int b = 2 * tid + k;
       if (b < B) {
@@ -280,48 +319,44 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const DecodePa
         }
         sm_len[b] = len;
         lu += (int64_t)p.Hkv * len;
-        lr += (int64_t)p.Hq * min(p.budget, len);
       }
     }
-    const int64_t pu = block_exclusive_scan(lu, sm_scan, &uoff_total);
-    const int64_t pr = block_exclusive_scan(lr, sm_scan, &roff_total);
-    int64_t au = pu, ar = pr;
+    const int64_t pu = block_exclusive_scan(lu, sm_scan, &U);
+    int64_t au = pu;
+    int same = 1;
     for (int k = 0; k < 2; ++k) {
       const int b = 2 * tid + k;
       if (b < B) {
         sm_uoff[b] = au;
-        sm_roff[b] = ar;
         au += (int64_t)p.Hkv * sm_len[b];
-        ar += (int64_t)p.Hq * min(p.budget, sm_len[b]);
+        same &= sm_len[b] == sm_len[0];
       }
     }
-    if (tid == 0) {
-      sm_uoff[B] = uoff_total;
-      sm_roff[B] = roff_total;
-    }
-    __syncthreads();
+    if (tid == 0) sm_uoff[B] = U;
+    uniform = __syncthreads_and(same);
   }
-  const int64_t U = uoff_total;
-  const int64_t u_lo = U > 0 ? range_begin(s, U, S) : 0;
-  const int64_t u_hi = U > 0 ? range_begin(s + 1, U, S) : 0;
+  // Blocks the units are split over: a multiple of the kv-head count when every
+  // sequence has the same length, so that no block straddles two kv heads.
+  const int heads = B * p.Hkv;
+  const int Sr = (uniform && heads <= S && U > 0) ? (S / heads) * heads : S;
+  const int64_t u_lo = (U > 0 && s < Sr) ? range_begin(s, U, Sr) : 0;
+  int64_t u_hi = (U > 0 && s < Sr) ? range_begin(s + 1, U, Sr) : 0;
+  if (u_hi - u_lo > p.range_cap) {  // never with the host's sizing; refuse rather than overrun
+    atomicOr(p.ctrl + 2, kErrInternal);
+    u_hi = u_lo;
+  }
 
   // ================================================================ phase 1
-  uint32_t gstage = 0;  // stages consumed so far by this block (same in every thread)
+  constexpr int kU = G <= 2 ? 4 : 2;  // code rows per thread per iteration, two iterations in flight
+  constexpr int kPerIt = kThreads * kU;
   for (int64_t u = u_lo; u < u_hi;) {
     const Segment seg = segment_at(u, u_lo, u_hi, sm_uoff, sm_len, B, p.Hkv);
-    const unsigned char* src = p.codes + ((int64_t)seg.hk * p.Nmax + seg.t0) * kCodeBytes;
-    const int64_t nst = (seg.len + kStageTokens - 1) / kStageTokens;
-    auto issue = [&](int64_t i) {
-      const uint32_t buf = (gstage + (uint32_t)i) % (uint32_t)nstages;
-      const int64_t rows = min((int64_t)kStageTokens, seg.len - i * kStageTokens);
-      const uint32_t bytes = (uint32_t)rows * kCodeBytes;
-      mbar_arrive_expect_tx(&sm_full[buf], bytes);
-      bulk_copy_g2s(sm_big + buf * kStageBytes, src + i * kStageBytes, bytes, &sm_full[buf]);
-    };
-    if (tid == 0) {
-      fence_proxy_async_smem();
-      for (int64_t i = 0; i < min(nst, (int64_t)nstages - 1); ++i) issue(i);
-    }
+    const uint8_t* crow = p.codes + ((int64_t)seg.hk * p.Nmax + seg.t0) * kCodeBytes;
+    const int seg_len = (int)seg.len;  // < 2^23 (checked by the host)
+    uint16_t* dseg = dbuf + seg.soff;
+    const int nit = (seg_len + kPerIt - 1) / kPerIt;
+    uint32_t ka[kU][kCodeWords], kb[kU][kCodeWords];
+    load_rows<kU>(ka, crow, 0, seg_len, tid);  // in flight while the query is encoded
     if (warp < G) {
       const int hq = seg.b * p.Hq + seg.kvh * G + warp;
       const uint32_t w = encode128_warp(p.q + (int64_t)hq * kDim, lane);
@@ -329,43 +364,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const DecodePa
     }
     for (int i = tid; i < G * kHistStride; i += kThreads) sm_work[i] = 0u;
     __syncthreads();
-
     uint32_t qw[G][kCodeWords];
 #pragma unroll
     for (int g = 0; g < G; ++g)
 #pragma unroll
       for (int w = 0; w < kCodeWords; ++w) qw[g][w] = sm_q[g * kCodeWords + w];
 
-    for (int64_t i = 0; i < nst; ++i) {
-      if (tid == 0 && i + nstages - 1 < nst) {
-        fence_proxy_async_smem();
-        issue(i + nstages - 1);
-      }
-      const uint32_t gs = gstage + (uint32_t)i;
-      const uint32_t buf = gs % (uint32_t)nstages;
-      if (!mbar_wait(&sm_full[buf], (gs / (uint32_t)nstages) & 1u, kMbarLimit)) atomicOr(p.ctrl + 2, kErrTimeout);
-      const unsigned char* stage = sm_big + buf * kStageBytes;
-#pragma unroll
-      for (int j = 0; j < kRowsPerThread; ++j) {
-        const int r = j * kThreads + tid;
-        const int64_t t = i * kStageTokens + r;
-        if (t < seg.len) {
-          const uint4* row = reinterpret_cast<const uint4*>(stage + r * kCodeBytes);
-          const uint4 a = row[0], c = row[1];
-          const uint32_t kc[kCodeWords] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
-          uint32_t e[kCodeWords];
-          key_odd_mask(kc, e);
-#pragma unroll
-          for (int g = 0; g < G; ++g) {
-            const int d = l1_distance(kc, e, qw[g]);
-            dbuf[(int64_t)g * dstride + seg.soff + t] = (uint16_t)d;
-            atomicAdd(&sm_work[g * kHistStride + d], 1u);
-          }
-        }
-      }
-      __syncthreads();
+    for (int it = 0; it < nit; it += 2) {
+      if (it + 1 < nit) load_rows<kU>(kb, crow, (it + 1) * kPerIt, seg_len, tid);
+      score_rows<G, kU>(ka, qw, it * kPerIt, seg_len, tid, dseg, dstride, sm_work);
+      if (it + 2 < nit) load_rows<kU>(ka, crow, (it + 2) * kPerIt, seg_len, tid);
+      if (it + 1 < nit) score_rows<G, kU>(kb, qw, (it + 1) * kPerIt, seg_len, tid, dseg, dstride, sm_work);
     }
-    gstage += (uint32_t)nst;
+    __syncthreads();
     for (int i = tid; i < G * kBins; i += kThreads) {
       const int g = i / kBins, d = i - g * kBins;
       p.hist[((int64_t)(s + seg.hk) * G + g) * kHistStride + d] = sm_work[g * kHistStride + d];
@@ -377,20 +388,22 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const DecodePa
   if (!grid_wait(p.ctrl, S, gen0, &sm_flag)) return;
 
   // ================================================================ phase 2
-  uint32_t* sm_cnt = sm_work;                                // [kWarps][kHistStride]
-  uint32_t* sm_rank = sm_work + kWarps * kHistStride;        // [kHistStride]
-  uint32_t* sm_round = sm_work + (kWarps + 1) * kHistStride; // [kHistStride]
-  uint32_t* cand = reinterpret_cast<uint32_t*>(sm_big);      // per-warp lists over the idle ring
-  const int cap_w = (int)(DecodeSmem::ring(nstages) / 4 / kWarps);
-  const int64_t round_tokens = (int64_t)kWarps * (cap_w - 32) / 8 * 8;
-  uint32_t* my_list = cand + warp * cap_w;
+  uint32_t* sm_cnt = sm_work;                          // [kWarps][kHistStride]
+  uint32_t* sm_rank = sm_work + kWarps * kHistStride;  // [kHistStride]
+  float* sm_state = reinterpret_cast<float*>(sm_work); // [2*kWarps][kPartial], after the gather
+  uint32_t* scr = sm_scratch + warp * kScratch;
+  const int half = p.row_cap / 2;
+  const int hw = tid >> 4, hl = tid & 15;
+  const float kScoreScale = 0.08838834764831845f * 1.4426950408889634f;  // log2(e)/sqrt(128)
+
   for (int64_t u = u_lo; u < u_hi;) {
     const Segment seg = segment_at(u, u_lo, u_hi, sm_uoff, sm_len, B, p.Hkv);
     const int64_t len_b = sm_len[seg.b];
     const int keff = (int)min((int64_t)p.budget, len_b);
+    const int seg_len = (int)seg.len, soff = (int)seg.soff;
     if (keff > 0) {
       if (warp == 0) {
-        const int n = list_blocks(owner_of(seg.head_u0, U, S), owner_of(seg.head_u0 + len_b - 1, U, S), U, S,
+        const int n = list_blocks(owner_of(seg.head_u0, U, Sr), owner_of(seg.head_u0 + len_b - 1, U, Sr), U, Sr,
                                   sm_list);
         if (lane == 0) sm_nlist = n;
       }
@@ -398,9 +411,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const DecodePa
       const int nlist = sm_nlist;
       const bool first_segment = sm_list[0] == s;
       const int64_t kv_base = (int64_t)seg.hk * p.Nmax;
+      // warp slices over 8-position groups of the segment's distances
+      const int a0 = soff, a1 = soff + seg_len;
+      const int grp0 = a0 >> 3, ngrp = ((a1 + 7) >> 3) - grp0;
+      const int gpw = (ngrp + kWarps - 1) / kWarps;
+      const int wg0 = grp0 + min(ngrp, warp * gpw), wg1 = grp0 + min(ngrp, (warp + 1) * gpw);
       for (int g = 0; g < G; ++g) {
         const int64_t hq = (int64_t)seg.b * p.Hq + seg.kvh * G + g;
         int32_t* idx_h = p.idx + hq * p.budget;
+        const uint16_t* drow = dbuf + (size_t)g * dstride;
         // ---- threshold and rank bases from the head's histograms
         int64_t H = 0, P = 0;
         if (tid < kBins) {
@@ -425,93 +444,250 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const DecodePa
           sm_rank[tid] = (uint32_t)(base + P);
         }
         __syncthreads();
-        const int T = sm_T;
-        const uint16_t* drow = dbuf + (int64_t)g * dstride;
-        // ---- rounds over slices of the segment, in index order
-        for (int64_t r0 = 0; r0 < seg.len; r0 += round_tokens) {
-          const int64_t a0 = seg.soff + r0, a1 = seg.soff + min(seg.len, r0 + round_tokens);
-          const int64_t grp0 = a0 >> 3, ngrp = ((a1 + 7) >> 3) - grp0;
-          const int64_t gpw = (ngrp + kWarps - 1) / kWarps;
-          const int64_t wg0 = grp0 + min(ngrp, (int64_t)warp * gpw), wg1 = grp0 + min(ngrp, (int64_t)(warp + 1) * gpw);
+        const uint32_t T = (uint32_t)sm_T;
+
+        float qf[8];
+        {
+          const uint4 qr = *reinterpret_cast<const uint4*>(p.q + hq * kDim + 8 * hl);
+          qf[0] = bf16_lo(qr.x) * kScoreScale; qf[1] = bf16_hi(qr.x) * kScoreScale;
+          qf[2] = bf16_lo(qr.y) * kScoreScale; qf[3] = bf16_hi(qr.y) * kScoreScale;
+          qf[4] = bf16_lo(qr.z) * kScoreScale; qf[5] = bf16_hi(qr.z) * kScoreScale;
+          qf[6] = bf16_lo(qr.w) * kScoreScale; qf[7] = bf16_hi(qr.w) * kScoreScale;
+        }
+        float m_run = -INFINITY, l_run = 0.0f, o[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) o[e] = 0.0f;
+
+        // sweeps of at most kMaxKept kept tokens (one sweep when budget <= kMaxKept)
+        for (int c0 = 0;; c0 += kMaxKept) {
           for (int i = tid; i < kWarps * kHistStride; i += kThreads) sm_cnt[i] = 0u;
           __syncthreads();
-          // compaction: tokens with D <= T, in index order, into this warp's list
-          int n_w = 0;
-          for (int64_t gb = wg0; gb < wg1; gb += 32) {
-            const int64_t grp = gb + lane;
-            uint4 v = make_uint4(0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu);
-            if (grp < wg1) v = *reinterpret_cast<const uint4*>(drow + grp * 8);
-            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-            uint32_t mask = 0;
+          // ---- pass 1: per-warp counts of the candidates (D <= T) per distance
+          int nlt = 0, neq = 0;
+          for (int gb = wg0; gb < wg1; gb += 32) {
+            const int grp = gb + lane;
+            uint32_t dv[8];
+            load_dist8(drow, grp, grp < wg1, dv);
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-              const int64_t pos = grp * 8 + e;
-              const uint32_t d = (w4[e >> 1] >> (16 * (e & 1))) & 0xFFFFu;
-              if (grp < wg1 && pos >= a0 && pos < a1 && d <= (uint32_t)T) mask |= 1u << e;
-            }
-            const int c = __popc(mask);
-            int incl = c;
-#pragma unroll
-            for (int o = 1; o < 32; o *= 2) {
-              const int y = __shfl_up_sync(0xffffffffu, incl, o);
-              if (lane >= o) incl += y;
-            }
-            const int total = __shfl_sync(0xffffffffu, incl, 31);
-            int at = n_w + incl - c;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              if (mask & (1u << e)) {
-                const uint32_t d = (w4[e >> 1] >> (16 * (e & 1))) & 0xFFFFu;
-                my_list[at++] = (uint32_t)(grp * 8 + e - seg.soff) << 9 | d;
+              const int pos = grp * 8 + e;
+              if (dv[e] <= T && pos >= a0 && pos < a1) {
+                atomicAdd(&sm_cnt[warp * kHistStride + dv[e]], 1u);
+                nlt += dv[e] < T;
+                neq += dv[e] == T;
               }
             }
-            n_w += total;
           }
-          // per-warp counts per distance, then exclusive prefix over the warps
-          for (int k = lane; k < n_w; k += 32) atomicAdd(&sm_cnt[warp * kHistStride + (my_list[k] & 511u)], 1u);
+#pragma unroll
+          for (int o2 = 16; o2 > 0; o2 /= 2) {
+            nlt += __shfl_xor_sync(0xffffffffu, nlt, o2);
+            neq += __shfl_xor_sync(0xffffffffu, neq, o2);
+          }
+          if (lane == 0) {
+            sm_wlt[warp] = nlt;
+            sm_weq[warp] = neq;
+          }
           __syncthreads();
-          if (tid <= T) {
+          if (tid <= (int)T) {  // exclusive prefix over the warps, per distance
             uint32_t run = 0;
             for (int w = 0; w < kWarps; ++w) {
               const uint32_t c = sm_cnt[w * kHistStride + tid];
               sm_cnt[w * kHistStride + tid] = run;
               run += c;
             }
-            sm_round[tid] = run;
           }
-          __syncthreads();
-          // placement, in index order within the warp's list
-          for (int k0 = 0; k0 < n_w; k0 += 32) {
-            const int k = k0 + lane;
-            const bool valid = k < n_w;
-            const uint32_t ent = valid ? my_list[k] : 0u;
-            const int d = (int)(ent & 511u);
-            const uint32_t m = __ballot_sync(0xffffffffu, valid);
-            uint32_t peers = 0;
-            if (valid) {
-              peers = __match_any_sync(m, d);
-              const uint32_t slot = sm_rank[d] + sm_cnt[warp * kHistStride + d] + __popc(peers & lt);
-              if (slot < (uint32_t)keff) {
-                const int64_t t = seg.t0 + (int64_t)(ent >> 9);
-                idx_h[slot] = (int32_t)t;
-                const uint16_t* kr = p.K + (kv_base + t) * kDim;
-                const uint16_t* vr = p.V + (kv_base + t) * kDim;
-                prefetch_l2_keep(kr);
-                prefetch_l2_keep(kr + 64);
-                prefetch_l2_keep(vr);
-                prefetch_l2_keep(vr + 64);
-              }
+          if (tid == 0) {  // kept tokens per warp: every D < T, and the ties at T within the quota
+            const int tie0 = (int)sm_rank[T];
+            int ties_before = 0, kept_before = 0;
+            for (int w = 0; w < kWarps; ++w) {
+              const int ties = min(max(keff - (tie0 + ties_before), 0), sm_weq[w]);
+              sm_wkept[w] = kept_before;
+              kept_before += sm_wlt[w] + ties;
+              ties_before += sm_weq[w];
             }
-            __syncwarp();
-            if (valid && (peers & lt) == 0u) sm_cnt[warp * kHistStride + d] += __popc(peers);
-            __syncwarp();
+            sm_kept_total = kept_before;
           }
           __syncthreads();
-          if (tid <= T) sm_rank[tid] += sm_round[tid];
+          const int kept_total = sm_kept_total;
+          // ---- pass 2: in index order, every candidate to its final slot
+          int kept_at = sm_wkept[warp];
+          for (int gb = wg0; gb < wg1; gb += 32) {
+            const int grp = gb + lane;
+            uint32_t dv[8];
+            load_dist8(drow, grp, grp < wg1, dv);
+            uint32_t mask = 0;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const int pos = grp * 8 + e;
+              if (dv[e] <= T && pos >= a0 && pos < a1) mask |= 1u << e;
+            }
+            const int c = __popc(mask);
+            if (__ballot_sync(0xffffffffu, c != 0) == 0u) continue;
+            int incl = c;
+#pragma unroll
+            for (int o2 = 1; o2 < 32; o2 *= 2) {
+              const int y = __shfl_up_sync(0xffffffffu, incl, o2);
+              if (lane >= o2) incl += y;
+            }
+            const int total = __shfl_sync(0xffffffffu, incl, 31);
+            int at = incl - c;
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              if (mask & (1u << e)) scr[at++] = (uint32_t)(grp * 8 + e - soff) << 9 | dv[e];
+            __syncwarp();
+            for (int k0 = 0; k0 < total; k0 += 32) {
+              const int k = k0 + lane;
+              const bool valid = k < total;
+              const uint32_t ent = valid ? scr[k] : 0u;
+              const uint32_t d = ent & 511u;
+              const uint32_t m = __ballot_sync(0xffffffffu, valid);
+              uint32_t peers = 0;
+              bool kept = false;
+              if (valid) {
+                peers = __match_any_sync(m, d);
+                const uint32_t slot = sm_rank[d] + sm_cnt[warp * kHistStride + d] + __popc(peers & lt);
+                if (slot < (uint32_t)keff) {
+                  kept = true;
+                  if (c0 == 0) idx_h[slot] = (int32_t)(seg.t0 + (int64_t)(ent >> 9));
+                }
+              }
+              const uint32_t kb = __ballot_sync(0xffffffffu, kept);
+              const int pos_k = kept_at + __popc(kb & lt);
+              if (kept && pos_k >= c0 && pos_k < c0 + kMaxKept) sm_kept[pos_k - c0] = (int32_t)(ent >> 9);
+              kept_at += __popc(kb);
+              __syncwarp();
+              if (valid && (peers & lt) == 0u) sm_cnt[warp * kHistStride + d] += __popc(peers);
+              __syncwarp();
+            }
+          }
           __syncthreads();
+          // ---- gather the listed kept rows, double-buffered halves of the staging area
+          const int n_list = max(0, min(kMaxKept, kept_total - c0));
+          const int nch = (n_list + half - 1) / half;
+          auto issue = [&](int ch) {
+            const int r0 = ch * half, n = min(half, n_list - r0);
+            unsigned char* buf = sm_rows + (size_t)(ch & 1) * half * kRowBytes;
+            for (int c = tid; c < n * 32; c += kThreads) {
+              const int row = c >> 5, piece = c & 31;
+              const int64_t t = seg.t0 + sm_kept[r0 + row];
+              const uint16_t* srcp = (piece < 16 ? p.K : p.V) + (kv_base + t) * kDim + (piece & 15) * 8;
+              cp_async16(buf + (size_t)row * kRowBytes + piece * 16, srcp);
+            }
+            cp_async_commit();
+          };
+          if (nch > 0) issue(0);
+          for (int ch = 0; ch < nch; ++ch) {
+            if (ch + 1 < nch) {
+              issue(ch + 1);
+              cp_async_wait<1>();
+            } else {
+              cp_async_wait<0>();
+            }
+            __syncthreads();
+            const int n = min(half, n_list - ch * half);
+            const unsigned char* buf = sm_rows + (size_t)(ch & 1) * half * kRowBytes;
+            // The trip count depends on the warp only, so both half-warps always
+            // reach the full-warp shuffles below together.
+            for (int rb = 2 * warp; rb < n; rb += 2 * kWarps) {
+              const int row = rb + (hw & 1);
+              const bool valid = row < n;
+              float sc = 0.0f;
+              uint4 vr = make_uint4(0, 0, 0, 0);
+              if (valid) {
+                const uint4 kr = *reinterpret_cast<const uint4*>(buf + (size_t)row * kRowBytes + 16 * hl);
+                vr = *reinterpret_cast<const uint4*>(buf + (size_t)row * kRowBytes + kDim * 2 + 16 * hl);
+                sc = qf[0] * bf16_lo(kr.x) + qf[1] * bf16_hi(kr.x) + qf[2] * bf16_lo(kr.y) + qf[3] * bf16_hi(kr.y) +
+                     qf[4] * bf16_lo(kr.z) + qf[5] * bf16_hi(kr.z) + qf[6] * bf16_lo(kr.w) + qf[7] * bf16_hi(kr.w);
+              }
+              sc += __shfl_xor_sync(0xffffffffu, sc, 8);
+              sc += __shfl_xor_sync(0xffffffffu, sc, 4);
+              sc += __shfl_xor_sync(0xffffffffu, sc, 2);
+              sc += __shfl_xor_sync(0xffffffffu, sc, 1);
+              if (!valid) continue;
+              const float m_new = fmaxf(m_run, sc);
+              const float corr = exp2f(m_run - m_new);
+              const float pr = exp2f(sc - m_new);
+              l_run = l_run * corr + pr;
+              const float vv[8] = {bf16_lo(vr.x), bf16_hi(vr.x), bf16_lo(vr.y), bf16_hi(vr.y),
+                                   bf16_lo(vr.z), bf16_hi(vr.z), bf16_lo(vr.w), bf16_hi(vr.w)};
+#pragma unroll
+              for (int e = 0; e < 8; ++e) o[e] = o[e] * corr + pr * vv[e];
+              m_run = m_new;
+            }
+            __syncthreads();
+          }
+          if (c0 + kMaxKept >= kept_total) break;
         }
         if (first_segment)
           for (int r = keff + tid; r < p.budget; r += kThreads) idx_h[r] = -1;
+        // ---- half-warp states -> this block's partial state for the query head
+        {
+          float* st = sm_state + hw * kPartial;
+          if (hl == 0) { st[0] = m_run; st[1] = l_run; }
+#pragma unroll
+          for (int e = 0; e < 8; ++e) st[4 + 8 * hl + e] = o[e];
+        }
+        __syncthreads();
+        float* part = p.partial + ((int64_t)(s + seg.hk) * G + g) * kPartial;
+        if (tid < kDim) {
+          float M = -INFINITY;
+          for (int k = 0; k < 2 * kWarps; ++k) M = fmaxf(M, sm_state[k * kPartial]);
+          float L = 0.0f, O = 0.0f;
+          if (M != -INFINITY) {
+            for (int k = 0; k < 2 * kWarps; ++k) {
+              const float* sk = sm_state + k * kPartial;
+              const float wgt = exp2f(sk[0] - M);  // 0 for a half-warp without rows
+              L += sk[1] * wgt;
+              O += sk[4 + tid] * wgt;
+            }
+          }
+          part[4 + tid] = O;
+          if (tid == 0) { part[0] = M; part[1] = L; }
+        }
+        __threadfence();
+        __syncthreads();
+        if (tid == 0) {
+          const uint32_t prev = atomicAdd(&p.head_done[hq], 1u);
+          sm_last = prev + 1u == (uint32_t)nlist;
+        }
+        __syncthreads();
+        if (sm_last) {  // every block of the head has published: merge
+          __threadfence();
+          if (tid < kDim) {
+            float M = -INFINITY;
+            for (int k0 = 0; k0 < nlist; k0 += 8) {
+              float mv[8];
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                mv[j] = k0 + j < nlist ? __ldcg(p.partial + ((int64_t)(sm_list[k0 + j] + seg.hk) * G + g) * kPartial)
+                                       : -INFINITY;
+#pragma unroll
+              for (int j = 0; j < 8; ++j) M = fmaxf(M, mv[j]);
+            }
+            float L = 0.0f, O = 0.0f;
+            for (int k0 = 0; k0 < nlist; k0 += 8) {
+              float mv[8], lv[8], ov[8];
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                const bool in = k0 + j < nlist;
+                const float* ps = p.partial + (in ? ((int64_t)(sm_list[k0 + j] + seg.hk) * G + g) * kPartial : 0);
+                mv[j] = in ? __ldcg(ps) : -INFINITY;
+                lv[j] = in ? __ldcg(ps + 1) : 0.0f;
+                ov[j] = in ? __ldcg(ps + 4 + tid) : 0.0f;
+              }
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                if (mv[j] == -INFINITY) continue;  // a block that kept no token of this head
+                const float wgt = exp2f(mv[j] - M);
+                L += lv[j] * wgt;
+                O += ov[j] * wgt;
+              }
+            }
+            p.out[hq * kDim + tid] = O / L;
+          }
+          if (tid == 0) p.head_done[hq] = 0u;
+        }
+        __syncthreads();
       }
     }
     u += seg.len;
@@ -522,160 +698,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const DecodePa
     if (min(p.budget, sm_len[b]) > 0) continue;
     for (int i = tid; i < kDim; i += kThreads) p.out[hq * kDim + i] = 0.0f;
     for (int r = tid; r < p.budget; r += kThreads) p.idx[hq * p.budget + r] = -1;
-  }
-
-  if (!grid_wait(p.ctrl, S, gen0 + 1u, &sm_flag)) return;
-
-  // ================================================================ phase 3
-  const int64_t R = roff_total;
-  const int64_t r_lo = R > 0 ? range_begin(s, R, S) : 0;
-  const int64_t r_hi = R > 0 ? range_begin(s + 1, R, S) : 0;
-  float* sm_state = reinterpret_cast<float*>(sm_work);   // [2*kWarps][kPartial]
-  const int hw = tid >> 4, hl = tid & 15;
-  const float kScoreScale = 0.08838834764831845f * 1.4426950408889634f;  // log2(e)/sqrt(128)
-  for (int64_t r = r_lo; r < r_hi;) {
-    const int b = find_batch(sm_roff, B, r);
-    const int keff = min(p.budget, sm_len[b]);
-    const int64_t rel = r - sm_roff[b];
-    const int h = (int)(rel / keff);
-    const int64_t j0 = rel - (int64_t)h * keff;
-    const int64_t head_r0 = sm_roff[b] + (int64_t)h * keff;
-    const int64_t slen = min(r_hi, head_r0 + keff) - r;
-    const int64_t hq = (int64_t)b * p.Hq + h;
-    const int kvh = h / G;
-    const int64_t len_b = sm_len[b];
-    const int64_t kv_base = ((int64_t)b * p.Hkv + kvh) * p.Nmax;
-
-    float qf[8];
-    {
-      const uint4 qr = *reinterpret_cast<const uint4*>(p.q + hq * kDim + 8 * hl);
-      qf[0] = bf16_lo(qr.x) * kScoreScale; qf[1] = bf16_hi(qr.x) * kScoreScale;
-      qf[2] = bf16_lo(qr.y) * kScoreScale; qf[3] = bf16_hi(qr.y) * kScoreScale;
-      qf[4] = bf16_lo(qr.z) * kScoreScale; qf[5] = bf16_hi(qr.z) * kScoreScale;
-      qf[6] = bf16_lo(qr.w) * kScoreScale; qf[7] = bf16_hi(qr.w) * kScoreScale;
-    }
-    float m_run = -INFINITY, l_run = 0.0f, o[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) o[e] = 0.0f;
-
-    const int32_t* idx_h = p.idx + hq * p.budget + j0;
-    for (int64_t c0 = 0; c0 < slen; c0 += p.row_cap) {
-      const int n = (int)min((int64_t)p.row_cap, slen - c0);
-      for (int i = tid; i < n; i += kThreads) {
-        int32_t t = __ldcg(idx_h + c0 + i);
-        if (t < 0 || t >= len_b) t = -1;  // never read outside the sequence
-        sm_rowidx[i] = t;
-      }
-      __syncthreads();
-      // every thread copies 16-byte pieces: 16 pieces of K then 16 of V per row
-      for (int c = tid; c < n * 32; c += kThreads) {
-        const int row = c >> 5, piece = c & 31;
-        const int32_t t = sm_rowidx[row];
-        if (t >= 0) {
-          const uint16_t* srcp = (piece < 16 ? p.K : p.V) + (kv_base + t) * kDim + (piece & 15) * 8;
-          cp_async16(sm_big + (size_t)row * kRowBytes + piece * 16, srcp);
-        }
-      }
-      cp_async_wait_all();
-      __syncthreads();
-      // The trip count depends on the warp only, so both half-warps always reach
-      // the full-warp shuffles below together.
-      for (int rb = 2 * warp; rb < n; rb += 2 * kWarps) {
-        const int row = rb + (hw & 1);
-        const bool valid = row < n && sm_rowidx[row] >= 0;
-        float sc = 0.0f;
-        uint4 vr = make_uint4(0, 0, 0, 0);
-        if (valid) {
-          const uint4 kr = *reinterpret_cast<const uint4*>(sm_big + (size_t)row * kRowBytes + 16 * hl);
-          vr = *reinterpret_cast<const uint4*>(sm_big + (size_t)row * kRowBytes + kDim * 2 + 16 * hl);
-          sc = qf[0] * bf16_lo(kr.x) + qf[1] * bf16_hi(kr.x) + qf[2] * bf16_lo(kr.y) + qf[3] * bf16_hi(kr.y) +
-               qf[4] * bf16_lo(kr.z) + qf[5] * bf16_hi(kr.z) + qf[6] * bf16_lo(kr.w) + qf[7] * bf16_hi(kr.w);
-        }
-        sc += __shfl_xor_sync(0xffffffffu, sc, 8);
-        sc += __shfl_xor_sync(0xffffffffu, sc, 4);
-        sc += __shfl_xor_sync(0xffffffffu, sc, 2);
-        sc += __shfl_xor_sync(0xffffffffu, sc, 1);
-        if (!valid) continue;
-        const float m_new = fmaxf(m_run, sc);
-        const float corr = exp2f(m_run - m_new);
-        const float pr = exp2f(sc - m_new);
-        l_run = l_run * corr + pr;
-        const float vv[8] = {bf16_lo(vr.x), bf16_hi(vr.x), bf16_lo(vr.y), bf16_hi(vr.y),
-                             bf16_lo(vr.z), bf16_hi(vr.z), bf16_lo(vr.w), bf16_hi(vr.w)};
-#pragma unroll
-        for (int e = 0; e < 8; ++e) o[e] = o[e] * corr + pr * vv[e];
-        m_run = m_new;
-      }
-      __syncthreads();
-    }
-    // half-warp states -> block partial
-    float* st = sm_state + hw * kPartial;
-    if (hl == 0) { st[0] = m_run; st[1] = l_run; }
-#pragma unroll
-    for (int e = 0; e < 8; ++e) st[4 + 8 * hl + e] = o[e];
-    if (warp == 0) {
-      const int n = list_blocks(owner_of(head_r0, R, S), owner_of(head_r0 + keff - 1, R, S), R, S, sm_list);
-      if (lane == 0) sm_nlist = n;
-    }
-    __syncthreads();
-    const int nlist = sm_nlist;
-    float* part = p.partial + (s + hq) * kPartial;
-    if (tid < kDim) {
-      float M = -INFINITY;
-      for (int k = 0; k < 2 * kWarps; ++k) M = fmaxf(M, sm_state[k * kPartial]);
-      float L = 0.0f, O = 0.0f;
-      for (int k = 0; k < 2 * kWarps; ++k) {
-        const float* sk = sm_state + k * kPartial;
-        const float wgt = exp2f(sk[0] - M);  // 0 for a half-warp without rows
-        L += sk[1] * wgt;
-        O += sk[4 + tid] * wgt;
-      }
-      part[4 + tid] = O;
-      if (tid == 0) { part[0] = M; part[1] = L; }
-    }
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) {
-      const uint32_t prev = atomicAdd(&p.head_done[hq], 1u);
-      sm_last = prev + 1u == (uint32_t)nlist;
-    }
-    __syncthreads();
-    if (sm_last) {
-      __threadfence();
-      if (tid < kDim) {
-        float M = -INFINITY;
-        for (int k0 = 0; k0 < nlist; k0 += 8) {
-          float mv[8];
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            mv[j] = k0 + j < nlist ? __ldcg(p.partial + (sm_list[k0 + j] + hq) * kPartial) : -INFINITY;
-#pragma unroll
-          for (int j = 0; j < 8; ++j) M = fmaxf(M, mv[j]);
-        }
-        float L = 0.0f, O = 0.0f;
-        for (int k0 = 0; k0 < nlist; k0 += 8) {
-          float mv[8], lv[8], ov[8];
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const bool in = k0 + j < nlist;
-            const float* ps = p.partial + (in ? (sm_list[k0 + j] + hq) * kPartial : 0);
-            mv[j] = in ? __ldcg(ps) : -INFINITY;
-            lv[j] = in ? __ldcg(ps + 1) : 0.0f;
-            ov[j] = in ? __ldcg(ps + 4 + tid) : 0.0f;
-          }
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const float wgt = exp2f(mv[j] - M);
-            L += lv[j] * wgt;
-            O += ov[j] * wgt;
-          }
-        }
-        p.out[hq * kDim + tid] = O / L;
-      }
-      if (tid == 0) p.head_done[hq] = 0u;
-    }
-    __syncthreads();
-    r += slen;
   }
 }
 

@@ -64,6 +64,7 @@ enum adamas_status {
 /* Bits of the device error word. */
 #define ADAMAS_DEVERR_SEQLEN 0x1u  /* a seq_lens entry was outside [0, Nmax]; it was clamped */
 #define ADAMAS_DEVERR_TIMEOUT 0x2u /* a grid-wide wait gave up; the step's outputs are invalid */
+#define ADAMAS_DEVERR_INTERNAL 0x4u /* a block's share exceeded its planned size; outputs are invalid */
 
 /* Static description of a status code (never NULL). */
 const char *adamas_status_string(int status);
