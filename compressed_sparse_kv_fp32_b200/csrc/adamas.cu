@@ -125,7 +125,7 @@ static int cuda_fail(cudaError_t e) {
 }
 
 // Shared memory a block can use beyond the kernels' static shared memory.
-constexpr size_t kStaticSmemReserve = 8192;
+constexpr size_t kStaticSmemReserve = 6144;  // static shared memory of the kernels + per-block system use
 
 static int device_info(DeviceInfo** out) {
   int dev = 0;
@@ -135,11 +135,15 @@ static int device_info(DeviceInfo** out) {
   std::lock_guard<std::mutex> lock(g_mutex);
   DeviceInfo& d = g_devices[dev];
   if (d.sms == 0) {
-    int sms = 0, optin = 0;
+    int sms = 0, optin = 0, per_sm = 0;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
-        (e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess)
+        (e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev)) != cudaSuccess)
       return cuda_fail(e);
-    d.smem_optin = (size_t)optin > kStaticSmemReserve ? (size_t)optin - kStaticSmemReserve : 0;
+    // dynamic shared memory of one decode block when kBlocksPerSM share an SM
+    size_t budget = (size_t)per_sm / kBlocksPerSM;
+    if (budget > (size_t)optin) budget = (size_t)optin;
+    d.smem_optin = budget > kStaticSmemReserve ? budget - kStaticSmemReserve : 0;
     d.sms = sms;
   }
   *out = &d;
@@ -171,7 +175,7 @@ static int ws_layout(int B, int Hq, int Hkv, int64_t Nmax, int budget, const Dev
   const int G = Hq / Hkv;
   const int64_t umax = (int64_t)B * Hkv * Nmax;
   int64_t want = (umax + 2047) / 2048;
-  const int max_blocks = dev.sms < kMaxBlocks ? dev.sms : kMaxBlocks;
+  const int max_blocks = dev.sms * kBlocksPerSM < kMaxBlocks ? dev.sms * kBlocksPerSM : kMaxBlocks;
   L->S = (int)(want < 1 ? 1 : (want > max_blocks ? max_blocks : want));
   L->range_cap = umax > 0 ? (umax + L->S - 1) / L->S : 1;
   // With equal lengths the kernel may split over a multiple of the kv-head count

@@ -47,12 +47,15 @@
 namespace adamas {
 
 constexpr int kThreads = 512;
+constexpr int kBlocksPerSM = 1;
 constexpr int kWarps = kThreads / 32;
+constexpr int kBatchPerThread = kMaxBatch / kThreads;
+constexpr int kBinsPerThread = (kBins + kThreads - 1) / kThreads;
 constexpr int kHistStride = 388;                     // >= kBins, multiple of 4
 constexpr int kPartial = 132;                        // m, l, pad, pad, o[128]
 constexpr uint32_t kRowBytes = 2 * kDim * 2;         // one K row + one V row (bf16)
 constexpr int kScratch = 256;                        // candidate entries per warp per 256-token group
-constexpr int kMaxKept = 2048;                       // kept tokens listed per sweep
+constexpr int kMaxKept = 1024;                       // kept tokens listed per sweep
 constexpr int kMaxRowsStaged = 256;
 constexpr int kMinRowsStaged = 32;
 constexpr int kMaxBlocks = 1024;
@@ -262,7 +265,7 @@ __device__ __forceinline__ void load_dist8(const uint16_t* drow, int grp, bool i
 // SMEM_D: the distances of the block's share live in shared memory (else in the
 // workspace).
 template <int G, bool SMEM_D>
-__global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(kThreads, kBlocksPerSM) decode_step_kernel(const DecodeParams p) {
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ int sm_flag;
   __shared__ int sm_T;
@@ -307,10 +310,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const DecodePa
   int64_t U;
   int uniform;
   {
-    // B <= kMaxBatch = 2 * kThreads: thread i owns batches 2i and 2i+1
+    // B <= kMaxBatch: thread i owns batches kBatchPerThread*i + k
     int64_t lu = 0;
-    for (int k = 0; k < 2; ++k) {
-      const int b = 2 * tid + k;
+    for (int k = 0; k < kBatchPerThread; ++k) {
+      const int b = kBatchPerThread * tid + k;
       if (b < B) {
         int32_t len = p.seq_lens[b];
         if (len < 0 || (int64_t)len > p.Nmax) {
@@ -324,8 +327,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const DecodePa
     const int64_t pu = block_exclusive_scan(lu, sm_scan, &U);
     int64_t au = pu;
     int same = 1;
-    for (int k = 0; k < 2; ++k) {
-      const int b = 2 * tid + k;
+    for (int k = 0; k < kBatchPerThread; ++k) {
+      const int b = kBatchPerThread * tid + k;
       if (b < B) {
         sm_uoff[b] = au;
         au += (int64_t)p.Hkv * sm_len[b];
@@ -420,28 +423,46 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const DecodePa
         const int64_t hq = (int64_t)seg.b * p.Hq + seg.kvh * G + g;
         int32_t* idx_h = p.idx + hq * p.budget;
         const uint16_t* drow = dbuf + (size_t)g * dstride;
-        // ---- threshold and rank bases from the head's histograms
-        int64_t H = 0, P = 0;
-        if (tid < kBins) {
-          for (int k0 = 0; k0 < nlist; k0 += 8) {
-            uint32_t v[8];
+        // ---- threshold and rank bases from the head's histograms; thread i owns
+        // the distances kBinsPerThread*i + k
+        int64_t H[kBinsPerThread], P[kBinsPerThread];
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-              v[j] = k0 + j < nlist
-                         ? __ldcg(&p.hist[((int64_t)(sm_list[k0 + j] + seg.hk) * G + g) * kHistStride + tid])
-                         : 0u;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              H += v[j];
-              if (k0 + j < nlist && sm_list[k0 + j] < s) P += v[j];
-            }
-          }
+        for (int k = 0; k < kBinsPerThread; ++k) {
+          H[k] = 0;
+          P[k] = 0;
         }
+        for (int k0 = 0; k0 < nlist; k0 += 8) {
+          uint32_t v[8][kBinsPerThread];
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+#pragma unroll
+            for (int k = 0; k < kBinsPerThread; ++k) {
+              const int d = kBinsPerThread * tid + k;
+              v[j][k] = (k0 + j < nlist && d < kBins)
+                            ? __ldcg(&p.hist[((int64_t)(sm_list[k0 + j] + seg.hk) * G + g) * kHistStride + d])
+                            : 0u;
+            }
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+#pragma unroll
+            for (int k = 0; k < kBinsPerThread; ++k) {
+              H[k] += v[j][k];
+              if (k0 + j < nlist && sm_list[k0 + j] < s) P[k] += v[j][k];
+            }
+        }
+        int64_t hsum = 0;
+#pragma unroll
+        for (int k = 0; k < kBinsPerThread; ++k) hsum += H[k];
         int64_t tot;
-        const int64_t base = block_exclusive_scan(H, sm_scan, &tot);
-        if (tid < kBins) {
-          if (base < keff && base + H >= keff) sm_T = tid;
-          sm_rank[tid] = (uint32_t)(base + P);
+        int64_t base = block_exclusive_scan(hsum, sm_scan, &tot);
+#pragma unroll
+        for (int k = 0; k < kBinsPerThread; ++k) {
+          const int d = kBinsPerThread * tid + k;
+          if (d < kBins) {
+            if (base < keff && base + H[k] >= keff) sm_T = d;
+            sm_rank[d] = (uint32_t)(base + P[k]);
+          }
+          base += H[k];
         }
         __syncthreads();
         const uint32_t T = (uint32_t)sm_T;
@@ -488,11 +509,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const DecodePa
             sm_weq[warp] = neq;
           }
           __syncthreads();
-          if (tid <= (int)T) {  // exclusive prefix over the warps, per distance
+          for (int d = tid; d <= (int)T; d += kThreads) {  // exclusive prefix over the warps, per distance
             uint32_t run = 0;
             for (int w = 0; w < kWarps; ++w) {
-              const uint32_t c = sm_cnt[w * kHistStride + tid];
-              sm_cnt[w * kHistStride + tid] = run;
+              const uint32_t c = sm_cnt[w * kHistStride + d];
+              sm_cnt[w * kHistStride + d] = run;
               run += c;
             }
           }
