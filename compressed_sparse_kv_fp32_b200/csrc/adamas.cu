@@ -65,6 +65,28 @@ __global__ void __launch_bounds__(kEncThreads) encode_keys_kernel(const uint16_t
   dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
 }
 
+// Small encodes (appending a few tokens): one warp per vector, so a call costs
+// one warp-level rotation instead of a thread walking 896 dependent adds.
+constexpr int kEncWarpThreads = 256;
+constexpr int64_t kEncWarpMaxVectors = 8192;
+
+__global__ void __launch_bounds__(kEncWarpThreads) encode_keys_warp_kernel(const uint16_t* __restrict__ K,
+                                                                           uint8_t* __restrict__ codes,
+                                                                           const int32_t* __restrict__ pos_begin,
+                                                                           int count, int Hkv, int64_t Nmax,
+                                                                           int64_t nvec) {
+  const int lane = threadIdx.x & 31;
+  const int64_t v = (int64_t)blockIdx.x * (kEncWarpThreads / 32) + (threadIdx.x >> 5);
+  if (v >= nvec) return;  // whole warp leaves together
+  const int64_t hk = v / count, r = v - hk * count;
+  const int b = (int)(hk / Hkv);
+  const int64_t pos = (pos_begin ? (int64_t)pos_begin[b] : 0) + r;
+  if (pos < 0 || pos >= Nmax) return;  // whole warp leaves together
+  const int64_t row = hk * Nmax + pos;
+  const uint32_t w = encode128_warp(K + row * kDim, lane);
+  if (lane < kCodeWords) reinterpret_cast<uint32_t*>(codes + row * kCodeBytes)[lane] = w;
+}
+
 // ------------------------------------------------------------------ distance dump (test entry point)
 constexpr int kScoreThreads = 256;
 constexpr int kScoreUnroll = 4;
@@ -155,6 +177,7 @@ struct WsLayout {
   int S;
   int64_t range_cap;
   bool smem_d;
+  bool stage_in_d;
   int row_cap;
   size_t smem;
 };
@@ -171,7 +194,6 @@ static int check_shape(int B, int Hq, int Hkv, int64_t Nmax, int d, int budget) 
 }
 
 static int ws_layout(int B, int Hq, int Hkv, int64_t Nmax, int budget, const DeviceInfo& dev, WsLayout* L) {
-  (void)budget;
   const int G = Hq / Hkv;
   const int64_t umax = (int64_t)B * Hkv * Nmax;
   int64_t want = (umax + 2047) / 2048;
@@ -194,7 +216,10 @@ static int ws_layout(int B, int Hq, int Hkv, int64_t Nmax, int budget, const Dev
   L->smem_d = fixed + dist + (size_t)kMinRowsStaged * kRowBytes <= dev.smem_optin;
   const size_t left = dev.smem_optin - fixed - (L->smem_d ? dist : 0);
   if (dev.smem_optin < fixed + (size_t)kMinRowsStaged * kRowBytes) return ADAMAS_ERR_UNSUPPORTED;
-  size_t rows = left / kRowBytes;
+  // Staging the gathered rows over the distance row keeps most of the SM's
+  // unified L1/shared storage as L1 for the code stream.
+  L->stage_in_d = L->smem_d && budget <= kMaxKept && DecodeSmem::dstride(L->range_cap) * 2 / kRowBytes >= 64;
+  size_t rows = L->stage_in_d ? kMinRowsStaged : left / kRowBytes;  // small fallback area for short segments
   if (rows > (size_t)kMaxRowsStaged) rows = kMaxRowsStaged;
   L->row_cap = (int)(rows & ~(size_t)1);
   L->smem = DecodeSmem::total(B, G, L->range_cap, L->smem_d, L->row_cap);
@@ -294,8 +319,16 @@ int adamas_encode_keys(const void* K, uint8_t* codes, const int32_t* pos_begin, 
   if (!K || !codes || !aligned(K, 16) || !aligned(codes, 32)) return ADAMAS_ERR_INVALID_ARG;
   if (pos_begin && !aligned(pos_begin, 4)) return ADAMAS_ERR_INVALID_ARG;
   const dim3 grid((unsigned)((count + kEncThreads - 1) / kEncThreads), (unsigned)(B * Hkv));
-  encode_keys_kernel<<<grid, kEncThreads, 0, (cudaStream_t)stream>>>(
-      static_cast<const uint16_t*>(K), codes, pos_begin, count, Hkv, Nmax);
+  const int64_t nvec = (int64_t)count * B * Hkv;
+  if (nvec <= kEncWarpMaxVectors) {
+    const int per_block = kEncWarpThreads / 32;
+    encode_keys_warp_kernel<<<(unsigned)((nvec + per_block - 1) / per_block), kEncWarpThreads, 0,
+                              (cudaStream_t)stream>>>(static_cast<const uint16_t*>(K), codes, pos_begin, count, Hkv,
+                                                      Nmax, nvec);
+  } else {
+    encode_keys_kernel<<<grid, kEncThreads, 0, (cudaStream_t)stream>>>(
+        static_cast<const uint16_t*>(K), codes, pos_begin, count, Hkv, Nmax);
+  }
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
   return ADAMAS_OK;
@@ -341,6 +374,7 @@ int adamas_decode_step(const void* q, const uint8_t* codes, const void* K, const
   prm.range_cap = L.range_cap;
   prm.smem_d = L.smem_d ? 1 : 0;
   prm.row_cap = L.row_cap;
+  prm.stage_in_d = L.stage_in_d ? 1 : 0;
 
   cudaStream_t st = (cudaStream_t)stream;
   switch (Hq / Hkv) {
@@ -491,6 +525,7 @@ extern "C" int adamas_decode_step_static(const void* q, const uint8_t* codes, co
   prm.range_cap = L.range_cap;
   prm.smem_d = L.smem_d ? 1 : 0;
   prm.row_cap = L.row_cap;
+  prm.stage_in_d = L.stage_in_d ? 1 : 0;
   switch (Hq / Hkv) {
     case 1: rc = launch_decode<1>(prm, L, *dev, st); break;
     case 2: rc = launch_decode<2>(prm, L, *dev, st); break;

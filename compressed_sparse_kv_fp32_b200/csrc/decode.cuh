@@ -13,8 +13,8 @@
 // heads so that no block straddles two heads); a block's share is handled as
 // "segments" (the part of one kv head inside the block's share).
 //   phase 1  per segment: encode the G query heads of the kv head, stream the
-//            packed code rows with 32-byte loads (each thread keeps the next rows
-//            in flight while it scores the current ones), keep the G distances of
+//            packed code rows with 32-byte loads (eight rows in flight per thread,
+//            256 KiB per block), keep the G distances of
 //            every token in shared memory and add them to one 385-bin histogram
 //            per query head; publish the histograms.
 //   -- grid-wide wait --
@@ -80,7 +80,8 @@ struct DecodeParams {
   int S;
   int64_t range_cap;    // >= units of any block
   int smem_d;           // distances kept in shared memory
-  int row_cap;          // K/V rows staged per gather buffer pair (even)
+  int row_cap;          // K/V rows of the dedicated gather staging (even; 0 with stage_in_d)
+  int stage_in_d;       // stage gathered rows over the finished distance row instead
 };
 
 // Shared-memory carve-up (bytes), shared with the host.
@@ -350,19 +351,21 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSM) decode_step_kernel(con
   }
 
   // ================================================================ phase 1
-  constexpr int kU = G <= 2 ? 4 : 2;  // code rows per thread per iteration, two iterations in flight
+  constexpr int kU = G <= 2 ? 8 : 4;  // code rows in flight per thread
   constexpr int kPerIt = kThreads * kU;
   for (int64_t u = u_lo; u < u_hi;) {
     const Segment seg = segment_at(u, u_lo, u_hi, sm_uoff, sm_len, B, p.Hkv);
     const uint8_t* crow = p.codes + ((int64_t)seg.hk * p.Nmax + seg.t0) * kCodeBytes;
     const int seg_len = (int)seg.len;  // < 2^23 (checked by the host)
     uint16_t* dseg = dbuf + seg.soff;
-    const int nit = (seg_len + kPerIt - 1) / kPerIt;
-    uint32_t ka[kU][kCodeWords], kb[kU][kCodeWords];
-    load_rows<kU>(ka, crow, 0, seg_len, tid);  // in flight while the query is encoded
+    // the query rows go first: loads issued after 128 KiB of code rows would
+    // queue behind them
+    uint2 qraw = make_uint2(0u, 0u);
+    if (warp < G) qraw = encode128_warp_load(p.q + ((int64_t)seg.b * p.Hq + seg.kvh * G + warp) * kDim, lane);
+    uint32_t kc[kU][kCodeWords];
+    load_rows<kU>(kc, crow, 0, seg_len, tid);  // in flight while the query is encoded
     if (warp < G) {
-      const int hq = seg.b * p.Hq + seg.kvh * G + warp;
-      const uint32_t w = encode128_warp(p.q + (int64_t)hq * kDim, lane);
+      const uint32_t w = encode128_warp_raw(qraw, lane);
       if (lane < kCodeWords) sm_q[warp * kCodeWords + lane] = w;
     }
     for (int i = tid; i < G * kHistStride; i += kThreads) sm_work[i] = 0u;
@@ -373,11 +376,9 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSM) decode_step_kernel(con
 #pragma unroll
       for (int w = 0; w < kCodeWords; ++w) qw[g][w] = sm_q[g * kCodeWords + w];
 
-    for (int it = 0; it < nit; it += 2) {
-      if (it + 1 < nit) load_rows<kU>(kb, crow, (it + 1) * kPerIt, seg_len, tid);
-      score_rows<G, kU>(ka, qw, it * kPerIt, seg_len, tid, dseg, dstride, sm_work);
-      if (it + 2 < nit) load_rows<kU>(ka, crow, (it + 2) * kPerIt, seg_len, tid);
-      if (it + 1 < nit) score_rows<G, kU>(kb, qw, (it + 1) * kPerIt, seg_len, tid, dseg, dstride, sm_work);
+    for (int base = 0; base < seg_len; base += kPerIt) {
+      if (base > 0) load_rows<kU>(kc, crow, base, seg_len, tid);
+      score_rows<G, kU>(kc, qw, base, seg_len, tid, dseg, dstride, sm_work);
     }
     __syncthreads();
     for (int i = tid; i < G * kBins; i += kThreads) {
@@ -395,7 +396,7 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSM) decode_step_kernel(con
   uint32_t* sm_rank = sm_work + kWarps * kHistStride;  // [kHistStride]
   float* sm_state = reinterpret_cast<float*>(sm_work); // [2*kWarps][kPartial], after the gather
   uint32_t* scr = sm_scratch + warp * kScratch;
-  const int half = p.row_cap / 2;
+
   const int hw = tid >> 4, hl = tid & 15;
   const float kScoreScale = 0.08838834764831845f * 1.4426950408889634f;  // log2(e)/sqrt(128)
 
@@ -423,6 +424,21 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSM) decode_step_kernel(con
         const int64_t hq = (int64_t)seg.b * p.Hq + seg.kvh * G + g;
         int32_t* idx_h = p.idx + hq * p.budget;
         const uint16_t* drow = dbuf + (size_t)g * dstride;
+        // gathered rows go over this segment's slice of the distance row just
+        // selected (free once its pass 2 is done; one sweep only) when it holds
+        // 64 rows or more, else to the dedicated area
+        unsigned char* stage = sm_rows;
+        int stage_cap = p.row_cap;
+        if (SMEM_D && p.stage_in_d) {
+          const size_t b0 = ((size_t)g * dstride + soff) * 2, b1 = b0 + (size_t)seg_len * 2;
+          const size_t a = (b0 + 127) / 128 * 128;
+          const int cap = b1 > a ? (int)min((size_t)kMaxRowsStaged, (b1 - a) / kRowBytes) & ~1 : 0;
+          if (cap >= 64) {
+            stage = reinterpret_cast<unsigned char*>(dbuf) + a;
+            stage_cap = cap;
+          }
+        }
+        const int half = stage_cap / 2;
         // ---- threshold and rank bases from the head's histograms; thread i owns
         // the distances kBinsPerThread*i + k
         int64_t H[kBinsPerThread], P[kBinsPerThread];
@@ -587,7 +603,7 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSM) decode_step_kernel(con
           const int nch = (n_list + half - 1) / half;
           auto issue = [&](int ch) {
             const int r0 = ch * half, n = min(half, n_list - r0);
-            unsigned char* buf = sm_rows + (size_t)(ch & 1) * half * kRowBytes;
+            unsigned char* buf = stage + (size_t)(ch & 1) * half * kRowBytes;
             for (int c = tid; c < n * 32; c += kThreads) {
               const int row = c >> 5, piece = c & 31;
               const int64_t t = seg.t0 + sm_kept[r0 + row];
@@ -606,7 +622,7 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSM) decode_step_kernel(con
             }
             __syncthreads();
             const int n = min(half, n_list - ch * half);
-            const unsigned char* buf = sm_rows + (size_t)(ch & 1) * half * kRowBytes;
+            const unsigned char* buf = stage + (size_t)(ch & 1) * half * kRowBytes;
             // The trip count depends on the warp only, so both half-warps always
             // reach the full-warp shuffles below together.
             for (int rb = 2 * warp; rb < n; rb += 2 * kWarps) {

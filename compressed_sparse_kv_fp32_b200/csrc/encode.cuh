@@ -53,22 +53,30 @@ __device__ __forceinline__ void fwht128_thread(float (&v)[kDim]) {
 }
 
 // Rotated values -> 8 little-endian words of packed codes.
+// With z = y + 0 (turns -0 into +0, leaves every other value unchanged) and
+// h = m/2, the three comparisons are sign bits of exact sums: [y < -h] is the
+// sign of z + h, [y < 0] the sign of z, [y < h] the sign of z - h (a nonzero
+// exact sum of two floats never rounds to zero, and x - x = +0).  The code is
+// 3 minus their sum, so its high bit is NOT sign(z) and its low bit is
+// NOT (sign(z + h) ^ sign(z) ^ sign(z - h)).  The bits are appended most
+// significant first with funnel shifts, inverted and byte-reversed at the end.
 __device__ __forceinline__ void bucket_pack_thread(const float (&y)[kDim], uint32_t (&w)[kCodeWords]) {
   float m = 0.0f;
 #pragma unroll
   for (int i = 0; i < kDim; ++i) m = fmaxf(m, fabsf(y[i]));
-  const float t0 = -0.5f * m, t2 = 0.5f * m;
+  const float h = 0.5f * m;
 #pragma unroll
   for (int i = 0; i < kCodeWords; ++i) {
-    uint32_t word = 0;
+    uint32_t acc = 0;
 #pragma unroll
-    for (int byte = 0; byte < 4; ++byte) {
-      const int e = 16 * i + 4 * byte;
-      const uint32_t b = code_of(y[e], t0, t2) << 6 | code_of(y[e + 1], t0, t2) << 4 |
-                         code_of(y[e + 2], t0, t2) << 2 | code_of(y[e + 3], t0, t2);
-      word |= b << (8 * byte);
+    for (int e = 0; e < 16; ++e) {
+      const float z = __fadd_rn(y[16 * i + e], 0.0f);
+      const uint32_t zb = __float_as_uint(z);
+      const uint32_t lo = __float_as_uint(__fadd_rn(z, h)) ^ zb ^ __float_as_uint(__fsub_rn(z, h));
+      acc = __funnelshift_l(zb, acc, 1);
+      acc = __funnelshift_l(lo, acc, 1);
     }
-    w[i] = word;
+    w[i] = __byte_perm(~acc, 0u, 0x0123);
   }
 }
 
@@ -77,8 +85,12 @@ __device__ __forceinline__ void bucket_pack_thread(const float (&y)[kDim], uint3
 // pairs lane L with lane L ^ (h / 4): the lane holding x[j] (bit h of j clear)
 // computes x[j] + x[j+h], the partner computes x[j] - x[j+h].
 // Returns, in every lane, packed code word (lane & 7).
-__device__ __forceinline__ uint32_t encode128_warp(const uint16_t* __restrict__ x, int lane) {
-  const uint2 raw = *reinterpret_cast<const uint2*>(x + 4 * lane);
+// `raw` holds the lane's four bf16 elements (loaded by encode128_warp_load).
+__device__ __forceinline__ uint2 encode128_warp_load(const uint16_t* __restrict__ x, int lane) {
+  return *reinterpret_cast<const uint2*>(x + 4 * lane);
+}
+
+__device__ __forceinline__ uint32_t encode128_warp_raw(uint2 raw, int lane) {
   float v0 = bf16_lo(raw.x), v1 = bf16_hi(raw.x), v2 = bf16_lo(raw.y), v3 = bf16_hi(raw.y);
   float a, b;
   // h = 1: (0,1) (2,3)
@@ -113,6 +125,10 @@ __device__ __forceinline__ uint32_t encode128_warp(const uint16_t* __restrict__ 
   w |= __shfl_xor_sync(0xffffffffu, w, 2);
   // lane 4i now holds word i; hand word (lane & 7) to every lane
   return __shfl_sync(0xffffffffu, w, 4 * (lane & 7));
+}
+
+__device__ __forceinline__ uint32_t encode128_warp(const uint16_t* __restrict__ x, int lane) {
+  return encode128_warp_raw(encode128_warp_load(x, lane), lane);
 }
 
 }  // namespace adamas
