@@ -106,38 +106,54 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(const uint16_t* __
   __syncthreads();
   int64_t len = seq_lens[b];
   len = len < 0 ? 0 : (len > Nmax ? Nmax : len);
-  uint32_t qw[G][kCodeWords];
+  uint32_t qw[G][kCodeWords], qm[G][kCodeWords];
 #pragma unroll
   for (int g = 0; g < G; ++g)
 #pragma unroll
-    for (int w = 0; w < kCodeWords; ++w) qw[g][w] = sq[g * kCodeWords + w];
+    for (int w = 0; w < kCodeWords; ++w) {
+      qw[g][w] = sq[g * kCodeWords + w];
+      qm[g][w] = query_mask(qw[g][w]);
+    }
   const int64_t first = (int64_t)blockIdx.x * kScoreThreads * kScoreUnroll;
 #pragma unroll
   for (int j = 0; j < kScoreUnroll; ++j) {
     const int64_t t = first + (int64_t)j * kScoreThreads + tid;
     if (t >= Nmax) break;
-    uint32_t kc[kCodeWords], e[kCodeWords];
+    uint32_t kc[kCodeWords], k1[kCodeWords];
     if (t < len) {
       ld_stream_v8(codes + ((int64_t)hk * Nmax + t) * kCodeBytes, kc);
-      key_odd_mask(kc, e);
+      key_shift(kc, k1);
     }
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-      const uint16_t d = t < len ? (uint16_t)l1_distance(kc, e, qw[g]) : (uint16_t)0xFFFF;
+      const uint16_t d = t < len ? (uint16_t)l1_distance(kc, k1, qw[g], qm[g]) : (uint16_t)0xFFFF;
       dist[((int64_t)b * Hq + kvh * G + g) * Nmax + t] = d;
     }
   }
 }
 
 // ------------------------------------------------------------------ host side
+constexpr int kMaxDevices = 64;
+constexpr int kMinTokensPerBlock = 2048;  // fewer tokens per block than this only when the context is short
+constexpr int kOccCache = 64;
+
+struct OccEntry {
+  const void* fn;
+  int cluster;
+  size_t smem;
+  int clusters;  // cudaOccupancyMaxActiveClusters
+};
+
 struct DeviceInfo {
   int sms = 0;
   size_t smem_optin = 0;
   bool attrs_set[2][kMaxGroup + 1] = {};
+  OccEntry occ[kOccCache] = {};
+  int n_occ = 0;
 };
 
 static std::mutex g_mutex;
-static DeviceInfo g_devices[64];
+static DeviceInfo g_devices[kMaxDevices];
 static thread_local cudaError_t g_last_cuda_error = cudaSuccess;
 
 // Record a failed CUDA call for adamas_last_error_string and map it to a status.
@@ -146,40 +162,104 @@ static int cuda_fail(cudaError_t e) {
   return ADAMAS_ERR_CUDA;
 }
 
-// Shared memory a block can use beyond the kernels' static shared memory.
-constexpr size_t kStaticSmemReserve = 6144;  // static shared memory of the kernels + per-block system use
+// Shared memory a block can use beyond the decode kernel's static shared memory.
+constexpr size_t kStaticSmemReserve = 2048;
 
-static int device_info(DeviceInfo** out) {
+static int device_info(DeviceInfo** out, int* dev_out = nullptr) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e);
-  if (dev < 0 || dev >= 64) return ADAMAS_ERR_UNSUPPORTED;
+  if (dev < 0 || dev >= kMaxDevices) return ADAMAS_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_mutex);
   DeviceInfo& d = g_devices[dev];
   if (d.sms == 0) {
-    int sms = 0, optin = 0, per_sm = 0;
+    int sms = 0, optin = 0;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
-        (e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess ||
-        (e = cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev)) != cudaSuccess)
+        (e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess)
       return cuda_fail(e);
-    // dynamic shared memory of one decode block when kBlocksPerSM share an SM
-    size_t budget = (size_t)per_sm / kBlocksPerSM;
-    if (budget > (size_t)optin) budget = (size_t)optin;
-    d.smem_optin = budget > kStaticSmemReserve ? budget - kStaticSmemReserve : 0;
+    d.smem_optin = (size_t)optin > kStaticSmemReserve ? (size_t)optin - kStaticSmemReserve : 0;
     d.sms = sms;
   }
   *out = &d;
+  if (dev_out) *dev_out = dev;
   return ADAMAS_OK;
 }
 
-struct WsLayout {
-  size_t ctrl, head_done, hist, partial, dspill, total;
-  int S;
-  int64_t range_cap;
-  bool smem_d;
-  bool stage_in_d;
-  int row_cap;
-  size_t smem;
+// One-time attributes of a decode kernel instance: the opt-in dynamic shared
+// memory and clusters of more than 8 blocks.
+static int kernel_attrs(DeviceInfo& dev, const void* fn, int G, bool smem_d) {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (dev.attrs_set[smem_d ? 1 : 0][G]) return ADAMAS_OK;
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dev.smem_optin);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  if (e != cudaSuccess) return cuda_fail(e);
+  dev.attrs_set[smem_d ? 1 : 0][G] = true;
+  return ADAMAS_OK;
+}
+
+// How many clusters of `cluster` blocks with `smem` bytes each can be resident at
+// once (cached per device).
+static int active_clusters(DeviceInfo& dev, const void* fn, int cluster, size_t smem, int* n) {
+  {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    for (int i = 0; i < dev.n_occ; ++i)
+      if (dev.occ[i].fn == fn && dev.occ[i].cluster == cluster && dev.occ[i].smem == smem) {
+        *n = dev.occ[i].clusters;
+        return ADAMAS_OK;
+      }
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)cluster);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)cluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int clusters = 0;
+  const cudaError_t e = cudaOccupancyMaxActiveClusters(&clusters, fn, &cfg);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();  // an unsupported cluster size is not sticky; treat it as 0
+    clusters = 0;
+  }
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (dev.n_occ < kOccCache) dev.occ[dev.n_occ++] = OccEntry{fn, cluster, smem, clusters};
+  *n = clusters;
+  return ADAMAS_OK;
+}
+
+template <int G, bool SMEM_D>
+static const void* decode_fn() {
+  return reinterpret_cast<const void*>(&decode_step_kernel<G, SMEM_D>);
+}
+
+static const void* decode_fn_for(int G, bool smem_d) {
+  switch (G) {
+    case 1: return smem_d ? decode_fn<1, true>() : decode_fn<1, false>();
+    case 2: return smem_d ? decode_fn<2, true>() : decode_fn<2, false>();
+    case 3: return smem_d ? decode_fn<3, true>() : decode_fn<3, false>();
+    case 4: return smem_d ? decode_fn<4, true>() : decode_fn<4, false>();
+    case 5: return smem_d ? decode_fn<5, true>() : decode_fn<5, false>();
+    case 6: return smem_d ? decode_fn<6, true>() : decode_fn<6, false>();
+    case 7: return smem_d ? decode_fn<7, true>() : decode_fn<7, false>();
+    case 8: return smem_d ? decode_fn<8, true>() : decode_fn<8, false>();
+    default: return nullptr;
+  }
+}
+
+// Launch plan and workspace layout of one decode step.
+struct Plan {
+  int G = 1;
+  int cluster = 1;   // blocks per (b, kv head)
+  int grid = 0;
+  int nstages = kMaxStages;
+  int dstride = 64;
+  bool smem_d = true;
+  size_t smem = 0;
+  size_t ctrl = 0, dspill = 0, total = 0;  // workspace offsets / size
 };
 
 static size_t align256(size_t x) { return (x + 255) / 256 * 256; }
@@ -193,75 +273,146 @@ static int check_shape(int B, int Hq, int Hkv, int64_t Nmax, int d, int budget) 
   return ADAMAS_OK;
 }
 
-static int ws_layout(int B, int Hq, int Hkv, int64_t Nmax, int budget, const DeviceInfo& dev, WsLayout* L) {
-  const int G = Hq / Hkv;
-  const int64_t umax = (int64_t)B * Hkv * Nmax;
-  int64_t want = (umax + 2047) / 2048;
-  const int max_blocks = dev.sms * kBlocksPerSM < kMaxBlocks ? dev.sms * kBlocksPerSM : kMaxBlocks;
-  L->S = (int)(want < 1 ? 1 : (want > max_blocks ? max_blocks : want));
-  L->range_cap = umax > 0 ? (umax + L->S - 1) / L->S : 1;
-  // With equal lengths the kernel may split over a multiple of the kv-head count
-  // (each block within one head): its shares are at most ceil(Nmax / (S / heads)).
-  const int64_t heads = (int64_t)B * Hkv;
-  if (heads > 0 && heads <= L->S) {
-    const int64_t per_head = L->S / heads;
-    const int64_t r2 = (Nmax + per_head - 1) / per_head;
-    if (r2 > L->range_cap) L->range_cap = r2;
+// Shared-memory layout for `cluster` blocks per head: distances in shared memory
+// with as many ring stages as fit, else in the workspace with a full ring.
+static bool layout_for(int G, int64_t Nmax, int cluster, size_t optin, Plan* P) {
+  const int64_t seg_cap = (Nmax + cluster - 1) / cluster;  // tokens of any block
+  if (seg_cap >= (int64_t(1) << 23)) return false;          // token offsets are packed in 23 bits
+  P->cluster = cluster;
+  P->dstride = (int)((seg_cap < 1 ? 1 : seg_cap) + 63) / 64 * 64;
+  for (int ns = kMaxStages; ns >= kMinStages; --ns) {
+    const size_t s = DecodeSmem::total(G, ns, P->dstride, true);
+    if (s <= optin) {
+      P->smem_d = true;
+      P->nstages = ns;
+      P->smem = s;
+      return true;
+    }
   }
-  if (L->range_cap >= (int64_t(1) << 23)) return ADAMAS_ERR_UNSUPPORTED;  // token offsets are packed in 23 bits
-  // Distances in shared memory when they fit beside the smallest gather staging;
-  // the staging then takes what is left (an even number of rows).
-  const size_t fixed = DecodeSmem::fixed(B, G);
-  const size_t dist = DecodeSmem::align128(DecodeSmem::dist(G, L->range_cap, true));
-  L->smem_d = fixed + dist + (size_t)kMinRowsStaged * kRowBytes <= dev.smem_optin;
-  const size_t left = dev.smem_optin - fixed - (L->smem_d ? dist : 0);
-  if (dev.smem_optin < fixed + (size_t)kMinRowsStaged * kRowBytes) return ADAMAS_ERR_UNSUPPORTED;
-  // Staging the gathered rows over the distance row keeps most of the SM's
-  // unified L1/shared storage as L1 for the code stream.
-  L->stage_in_d = L->smem_d && budget <= kMaxKept && DecodeSmem::dstride(L->range_cap) * 2 / kRowBytes >= 64;
-  size_t rows = L->stage_in_d ? kMinRowsStaged : left / kRowBytes;  // small fallback area for short segments
-  if (rows > (size_t)kMaxRowsStaged) rows = kMaxRowsStaged;
-  L->row_cap = (int)(rows & ~(size_t)1);
-  L->smem = DecodeSmem::total(B, G, L->range_cap, L->smem_d, L->row_cap);
-  if (L->smem > dev.smem_optin) return ADAMAS_ERR_UNSUPPORTED;
+  for (int ns = kMaxStages; ns >= kMinStages; --ns) {
+    const size_t s = DecodeSmem::total(G, ns, P->dstride, false);
+    if (s <= optin) {
+      P->smem_d = false;
+      P->nstages = ns;
+      P->smem = s;
+      return true;
+    }
+  }
+  return false;
+}
+
+// Cluster size: the largest that keeps every cluster resident at once (one
+// wave), at most one block per SM in total, and at least kMinTokensPerBlock
+// tokens per block; 1 when even single blocks need several waves.
+static int make_plan(int B, int Hq, int Hkv, int64_t Nmax, DeviceInfo& dev, Plan* P) {
+  const int G = Hq / Hkv;
+  const int heads = B * Hkv;
+  P->G = G;
+  int want = heads > 0 ? dev.sms / heads : 1;
+  const int64_t by_len = (Nmax + kMinTokensPerBlock - 1) / kMinTokensPerBlock;
+  if ((int64_t)want > by_len) want = (int)by_len;
+  if (want > kMaxCluster) want = kMaxCluster;
+  if (want < 1) want = 1;
+  bool found = false;
+  for (int c = want; c >= 1 && !found; --c) {
+    Plan t = *P;
+    if (!layout_for(G, Nmax, c, dev.smem_optin, &t)) continue;
+    const void* fn = decode_fn_for(G, t.smem_d);
+    int rc = kernel_attrs(dev, fn, G, t.smem_d);
+    if (rc != ADAMAS_OK) return rc;
+    int n = 0;
+    if ((rc = active_clusters(dev, fn, c, t.smem, &n)) != ADAMAS_OK) return rc;
+    if (n >= 1 && (n >= heads || c == 1)) {
+      *P = t;
+      found = true;
+    }
+  }
+  if (!found) return ADAMAS_ERR_UNSUPPORTED;
+  P->grid = heads * P->cluster;
   size_t off = 0;
-  L->ctrl = off;      off += align256(64 * sizeof(uint32_t));
-  L->head_done = off; off += align256((size_t)B * Hq * sizeof(uint32_t));
-  L->hist = off;      off += align256((size_t)(L->S + B * Hkv) * G * kHistStride * sizeof(uint32_t));
-  L->partial = off;   off += align256((size_t)(L->S + B * Hkv) * G * kPartial * sizeof(float));
-  L->dspill = off;
-  off += L->smem_d ? 0 : align256((size_t)L->S * G * DecodeSmem::dstride(L->range_cap) * sizeof(uint16_t));
-  L->total = off;
+  P->ctrl = off;   off += align256(64 * sizeof(uint32_t));
+  P->dspill = off;
+  off += P->smem_d ? 0 : align256((size_t)P->grid * G * P->dstride * sizeof(uint16_t));
+  P->total = off;
   return ADAMAS_OK;
 }
 
 static bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
 
 template <int G>
-static int launch_decode(const DecodeParams& prm, const WsLayout& L, DeviceInfo& dev, cudaStream_t stream) {
-  auto kernel = prm.smem_d ? decode_step_kernel<G, true> : decode_step_kernel<G, false>;
-  {
-    std::lock_guard<std::mutex> lock(g_mutex);
-    if (!dev.attrs_set[prm.smem_d ? 1 : 0][G]) {
-      const cudaError_t e =
-          cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dev.smem_optin);
-      if (e != cudaSuccess) return cuda_fail(e);
-      dev.attrs_set[prm.smem_d ? 1 : 0][G] = true;
-    }
-  }
+static int launch_decode(const DecodeParams& prm, const Plan& P, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)L.S);
+  cfg.gridDim = dim3((unsigned)P.grid);
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = L.smem;
+  cfg.dynamicSmemBytes = P.smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeCooperative;
-  attr[0].val.cooperative = 1;
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)P.cluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, prm);
+  const cudaError_t e = P.smem_d ? cudaLaunchKernelEx(&cfg, decode_step_kernel<G, true>, prm)
+                                 : cudaLaunchKernelEx(&cfg, decode_step_kernel<G, false>, prm);
   if (e != cudaSuccess) return cuda_fail(e);
   return ADAMAS_OK;
+}
+
+// Argument checks shared by both decode entry points (before anything is enqueued).
+static int check_decode_args(const void* q, const uint8_t* codes, const void* K, const void* V,
+                             const int32_t* seq_lens, int B, int Hq, int Hkv, int64_t Nmax, int d, int budget,
+                             const float* out, const int32_t* idx) {
+  int rc = check_shape(B, Hq, Hkv, Nmax, d, budget);
+  if (rc != ADAMAS_OK) return rc;
+  if (B == 0) return ADAMAS_OK;
+  if (!q || !seq_lens || !out || (budget > 0 && !idx)) return ADAMAS_ERR_INVALID_ARG;
+  if (Nmax > 0 && (!codes || !K || !V)) return ADAMAS_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(codes, 32) || !aligned(K, 16) || !aligned(V, 16) || !aligned(out, 16) ||
+      !aligned(idx, 4) || !aligned(seq_lens, 4))
+    return ADAMAS_ERR_INVALID_ARG;
+  return ADAMAS_OK;
+}
+
+// Enqueue the decode kernel with its scratch at `ws` (laid out by `P`).
+static int enqueue_decode(const void* q, const uint8_t* codes, const void* K, const void* V,
+                          const int32_t* seq_lens, int B, int Hq, int Hkv, int64_t Nmax, int budget, float* out,
+                          int32_t* idx, unsigned char* ws, const Plan& P, cudaStream_t st) {
+  DecodeParams prm;
+  prm.q = static_cast<const uint16_t*>(q);
+  prm.codes = codes;
+  prm.K = static_cast<const uint16_t*>(K);
+  prm.V = static_cast<const uint16_t*>(V);
+  prm.seq_lens = seq_lens;
+  prm.out = out;
+  prm.idx = idx;
+  prm.err = reinterpret_cast<uint32_t*>(ws + P.ctrl) + 2;
+  prm.dglobal = P.smem_d ? nullptr : reinterpret_cast<uint16_t*>(ws + P.dspill);
+  prm.B = B;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.Nmax = Nmax;
+  prm.budget = budget;
+  prm.cluster = P.cluster;
+  prm.nstages = P.nstages;
+  prm.dstride = P.dstride;
+  int rc;
+  switch (P.G) {
+    case 1: rc = launch_decode<1>(prm, P, st); break;
+    case 2: rc = launch_decode<2>(prm, P, st); break;
+    case 3: rc = launch_decode<3>(prm, P, st); break;
+    case 4: rc = launch_decode<4>(prm, P, st); break;
+    case 5: rc = launch_decode<5>(prm, P, st); break;
+    case 6: rc = launch_decode<6>(prm, P, st); break;
+    case 7: rc = launch_decode<7>(prm, P, st); break;
+    case 8: rc = launch_decode<8>(prm, P, st); break;
+    default: rc = ADAMAS_ERR_UNSUPPORTED;
+  }
+  if (rc == ADAMAS_OK) {
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) rc = cuda_fail(e);
+  }
+  return rc;
 }
 
 template <int G>
@@ -288,7 +439,7 @@ const char* adamas_status_string(int status) {
   }
 }
 
-int adamas_version(void) { return 100; }
+int adamas_version(void) { return 200; }
 
 const char* adamas_last_error_string(void) {
   return g_last_cuda_error == cudaSuccess ? "no CUDA error" : cudaGetErrorString(g_last_cuda_error);
@@ -298,9 +449,9 @@ size_t adamas_workspace_bytes(int B, int Hq, int Hkv, int64_t Nmax, int d, int b
   if (check_shape(B, Hq, Hkv, Nmax, d, budget) != ADAMAS_OK) return 0;
   DeviceInfo* dev = nullptr;
   if (device_info(&dev) != ADAMAS_OK) return 0;
-  WsLayout L;
-  if (ws_layout(B, Hq, Hkv, Nmax, budget, *dev, &L) != ADAMAS_OK) return 0;
-  return L.total;
+  Plan P;
+  if (make_plan(B, Hq, Hkv, Nmax, *dev, &P) != ADAMAS_OK) return 0;
+  return P.total;
 }
 
 int adamas_workspace_init(void* workspace, size_t workspace_bytes, adamas_stream_t stream) {
@@ -337,62 +488,15 @@ int adamas_encode_keys(const void* K, uint8_t* codes, const int32_t* pos_begin, 
 int adamas_decode_step(const void* q, const uint8_t* codes, const void* K, const void* V, const int32_t* seq_lens,
                        int B, int Hq, int Hkv, int64_t Nmax, int d, int budget, float* out, int32_t* idx,
                        void* workspace, size_t workspace_bytes, adamas_stream_t stream) {
-  int rc = check_shape(B, Hq, Hkv, Nmax, d, budget);
-  if (rc != ADAMAS_OK) return rc;
-  if (B == 0) return ADAMAS_OK;
-  if (!q || !seq_lens || !out || (budget > 0 && !idx)) return ADAMAS_ERR_INVALID_ARG;
-  if (Nmax > 0 && (!codes || !K || !V)) return ADAMAS_ERR_INVALID_ARG;
-  if (!aligned(q, 16) || !aligned(codes, 32) || !aligned(K, 16) || !aligned(V, 16) || !aligned(out, 16) ||
-      !aligned(idx, 4) || !aligned(seq_lens, 4))
-    return ADAMAS_ERR_INVALID_ARG;
+  int rc = check_decode_args(q, codes, K, V, seq_lens, B, Hq, Hkv, Nmax, d, budget, out, idx);
+  if (rc != ADAMAS_OK || B == 0) return rc;
   DeviceInfo* dev = nullptr;
   if ((rc = device_info(&dev)) != ADAMAS_OK) return rc;
-  WsLayout L;
-  if ((rc = ws_layout(B, Hq, Hkv, Nmax, budget, *dev, &L)) != ADAMAS_OK) return rc;
-  if (!workspace || workspace_bytes < L.total || !aligned(workspace, 16)) return ADAMAS_ERR_WORKSPACE;
-
-  unsigned char* ws = static_cast<unsigned char*>(workspace);
-  DecodeParams prm;
-  prm.q = static_cast<const uint16_t*>(q);
-  prm.codes = codes;
-  prm.K = static_cast<const uint16_t*>(K);
-  prm.V = static_cast<const uint16_t*>(V);
-  prm.seq_lens = seq_lens;
-  prm.out = out;
-  prm.idx = idx;
-  prm.ctrl = reinterpret_cast<uint32_t*>(ws + L.ctrl);
-  prm.head_done = reinterpret_cast<uint32_t*>(ws + L.head_done);
-  prm.hist = reinterpret_cast<uint32_t*>(ws + L.hist);
-  prm.partial = reinterpret_cast<float*>(ws + L.partial);
-  prm.dglobal = L.smem_d ? nullptr : reinterpret_cast<uint16_t*>(ws + L.dspill);
-  prm.B = B;
-  prm.Hq = Hq;
-  prm.Hkv = Hkv;
-  prm.Nmax = Nmax;
-  prm.budget = budget;
-  prm.S = L.S;
-  prm.range_cap = L.range_cap;
-  prm.smem_d = L.smem_d ? 1 : 0;
-  prm.row_cap = L.row_cap;
-  prm.stage_in_d = L.stage_in_d ? 1 : 0;
-
-  cudaStream_t st = (cudaStream_t)stream;
-  switch (Hq / Hkv) {
-    case 1: rc = launch_decode<1>(prm, L, *dev, st); break;
-    case 2: rc = launch_decode<2>(prm, L, *dev, st); break;
-    case 3: rc = launch_decode<3>(prm, L, *dev, st); break;
-    case 4: rc = launch_decode<4>(prm, L, *dev, st); break;
-    case 5: rc = launch_decode<5>(prm, L, *dev, st); break;
-    case 6: rc = launch_decode<6>(prm, L, *dev, st); break;
-    case 7: rc = launch_decode<7>(prm, L, *dev, st); break;
-    case 8: rc = launch_decode<8>(prm, L, *dev, st); break;
-    default: rc = ADAMAS_ERR_UNSUPPORTED;
-  }
-  if (rc == ADAMAS_OK) {
-    const cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) rc = cuda_fail(e);
-  }
-  return rc;
+  Plan P;
+  if ((rc = make_plan(B, Hq, Hkv, Nmax, *dev, &P)) != ADAMAS_OK) return rc;
+  if (!workspace || workspace_bytes < P.total || !aligned(workspace, 16)) return ADAMAS_ERR_WORKSPACE;
+  return enqueue_decode(q, codes, K, V, seq_lens, B, Hq, Hkv, Nmax, budget, out, idx,
+                        static_cast<unsigned char*>(workspace), P, (cudaStream_t)stream);
 }
 
 int adamas_score(const void* q, const uint8_t* codes, const int32_t* seq_lens, int B, int Hq, int Hkv, int64_t Nmax,
@@ -454,7 +558,7 @@ constexpr size_t kStaticScratchBytes = size_t(4) << 20;  // 4 MiB on every devic
 static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
 static std::mutex g_static_mutex;
-static void* g_static_scratch_ptr[64] = {};
+static void* g_static_scratch_ptr[kMaxDevices] = {};
 
 // Device address of g_static_scratch on the current device.  In host code the
 // array's name is only a host-side stand-in, so the address is looked up once
@@ -463,7 +567,7 @@ static int static_scratch(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e);
-  if (dev < 0 || dev >= 64) return ADAMAS_ERR_UNSUPPORTED;
+  if (dev < 0 || dev >= kMaxDevices) return ADAMAS_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_static_mutex);
   if (!g_static_scratch_ptr[dev]) {
     void* p = nullptr;
@@ -480,66 +584,20 @@ static int static_scratch(void** out) {
 extern "C" int adamas_decode_step_static(const void* q, const uint8_t* codes, const void* K, const void* V,
                                          const int32_t* seq_lens, int B, int Hq, int Hkv, int64_t Nmax, int d,
                                          int budget, float* out, int32_t* idx, adamas_stream_t stream) {
-  int rc = check_shape(B, Hq, Hkv, Nmax, d, budget);
-  if (rc != ADAMAS_OK) return rc;
-  if (B == 0) return ADAMAS_OK;
-  if (!q || !seq_lens || !out || (budget > 0 && !idx)) return ADAMAS_ERR_INVALID_ARG;
-  if (Nmax > 0 && (!codes || !K || !V)) return ADAMAS_ERR_INVALID_ARG;
-  if (!aligned(q, 16) || !aligned(codes, 32) || !aligned(K, 16) || !aligned(V, 16) || !aligned(out, 16) ||
-      !aligned(idx, 4) || !aligned(seq_lens, 4))
-    return ADAMAS_ERR_INVALID_ARG;
+  int rc = check_decode_args(q, codes, K, V, seq_lens, B, Hq, Hkv, Nmax, d, budget, out, idx);
+  if (rc != ADAMAS_OK || B == 0) return rc;
   DeviceInfo* dev = nullptr;
   if ((rc = device_info(&dev)) != ADAMAS_OK) return rc;
-  WsLayout L;
-  if ((rc = ws_layout(B, Hq, Hkv, Nmax, budget, *dev, &L)) != ADAMAS_OK) return rc;
-  if (L.total > kStaticScratchBytes) return ADAMAS_ERR_WORKSPACE;  // sizes beyond the fixed scratch
+  Plan P;
+  if ((rc = make_plan(B, Hq, Hkv, Nmax, *dev, &P)) != ADAMAS_OK) return rc;
+  if (P.total > kStaticScratchBytes) return ADAMAS_ERR_WORKSPACE;  // sizes beyond the fixed scratch
   void* scratch = nullptr;
   if ((rc = static_scratch(&scratch)) != ADAMAS_OK) return rc;
-
-  // The scratch keeps whatever the previous call left; the grid-wait counters,
-  // the error word and the per-head tickets must start at zero.
+  // The scratch keeps whatever the previous call left; the error word must start
+  // at zero.
   cudaStream_t st = (cudaStream_t)stream;
-  cudaError_t e = cudaMemsetAsync(scratch, 0, L.hist, st);
+  const cudaError_t e = cudaMemsetAsync(scratch, 0, P.dspill, st);
   if (e != cudaSuccess) return cuda_fail(e);
-
-  unsigned char* ws = static_cast<unsigned char*>(scratch);
-  DecodeParams prm;
-  prm.q = static_cast<const uint16_t*>(q);
-  prm.codes = codes;
-  prm.K = static_cast<const uint16_t*>(K);
-  prm.V = static_cast<const uint16_t*>(V);
-  prm.seq_lens = seq_lens;
-  prm.out = out;
-  prm.idx = idx;
-  prm.ctrl = reinterpret_cast<uint32_t*>(ws + L.ctrl);
-  prm.head_done = reinterpret_cast<uint32_t*>(ws + L.head_done);
-  prm.hist = reinterpret_cast<uint32_t*>(ws + L.hist);
-  prm.partial = reinterpret_cast<float*>(ws + L.partial);
-  prm.dglobal = L.smem_d ? nullptr : reinterpret_cast<uint16_t*>(ws + L.dspill);
-  prm.B = B;
-  prm.Hq = Hq;
-  prm.Hkv = Hkv;
-  prm.Nmax = Nmax;
-  prm.budget = budget;
-  prm.S = L.S;
-  prm.range_cap = L.range_cap;
-  prm.smem_d = L.smem_d ? 1 : 0;
-  prm.row_cap = L.row_cap;
-  prm.stage_in_d = L.stage_in_d ? 1 : 0;
-  switch (Hq / Hkv) {
-    case 1: rc = launch_decode<1>(prm, L, *dev, st); break;
-    case 2: rc = launch_decode<2>(prm, L, *dev, st); break;
-    case 3: rc = launch_decode<3>(prm, L, *dev, st); break;
-    case 4: rc = launch_decode<4>(prm, L, *dev, st); break;
-    case 5: rc = launch_decode<5>(prm, L, *dev, st); break;
-    case 6: rc = launch_decode<6>(prm, L, *dev, st); break;
-    case 7: rc = launch_decode<7>(prm, L, *dev, st); break;
-    case 8: rc = launch_decode<8>(prm, L, *dev, st); break;
-    default: rc = ADAMAS_ERR_UNSUPPORTED;
-  }
-  if (rc == ADAMAS_OK) {
-    e = cudaGetLastError();
-    if (e != cudaSuccess) rc = cuda_fail(e);
-  }
-  return rc;
+  return enqueue_decode(q, codes, K, V, seq_lens, B, Hq, Hkv, Nmax, budget, out, idx,
+                        static_cast<unsigned char*>(scratch), P, st);
 }

@@ -60,6 +60,11 @@ TINY = [
     (1, 8, 1, 300, [300], 17),
     (4, 12, 4, 129, [129, 1, 128, 64], 32),
     (1, 3, 1, 2048, [2047], 2048),
+    # 16 blocks per head, one head shorter than the cluster (blocks without tokens)
+    (2, 2, 2, 40000, [5, 40000], 16),
+    (1, 1, 1, 40000, [39999], 3000),
+    # distances too many for shared memory: they go through the workspace
+    (1, 8, 1, 200000, [200000], 512),
 ]
 
 
