@@ -11,33 +11,42 @@
 // the cluster owns the tokens [r*len/C, (r+1)*len/C) of the head.  Nothing is
 // exchanged through global memory: the blocks of a head share their histograms
 // and partial softmax states through distributed shared memory, so the step has
-// no grid-wide wait and no cross-cluster dependency.
+// no grid-wide wait and no dependency between clusters.
 //   phase 1  one warp streams the block's packed code rows into a ring of 32 KiB
 //            shared-memory stages with bulk asynchronous copies (one full and one
 //            empty mbarrier per stage); sixteen warps encode the G query heads of
 //            the kv head, then score every row against them (exact L1, two rows
 //            per thread per stage), keep the G distances of every token (shared
 //            memory, or the workspace when they do not fit) and count them in one
-//            385-bin histogram per query head.
+//            385-bin histogram per query head.  They also list the tokens that
+//            can still be selected: a further warp keeps reading the histograms
+//            of the whole cluster so far and publishes the smallest distance B
+//            with at least k_eff tokens at or below it -- the final threshold of
+//            the head can only be <= B -- and only tokens with D <= B are listed.
+//            When the cluster's histograms fit, every block then writes its own
+//            into a table in each peer.
 //   -- cluster barrier --
-//   phase 2  per query head: the C histograms (read from the peers' shared
-//            memory) give the threshold T with count(D < T) < k_eff <= count(D <= T)
-//            and, for every distance d, the number of tokens of the head with a
-//            smaller distance plus the number of tokens with distance d in
-//            lower-ranked blocks.  Pass 1: each warp counts, per distance, the
-//            tokens of its slice with D <= T.  Pass 2: each warp scans its slice
-//            again in index order and puts every candidate straight at its final
-//            slot of the (D, index)-ordered output: slot = #smaller D in the head
-//            + #equal D in lower blocks + #equal D in lower warps + #equal D in
-//            lower lanes (a warp match).  Slots >= k_eff are dropped, which keeps
-//            ties at T for the lowest indices.  The kept rows are then gathered
-//            straight into registers (each half-warp keeps four K and four V rows
-//            in flight) and folded into an online-softmax state per half-warp;
-//            the states become one partial (m, l, o) per query head and block.
+//   phase 2  per query head: the C histograms give the threshold T with
+//            count(D < T) < k_eff <= count(D <= T) and, for every distance d, the
+//            rank base = #tokens of the head with a smaller distance + #tokens
+//            with distance d in lower-ranked blocks.  Every token with D < T is
+//            kept; of the ties D == T this block keeps its first k_eff - base(T)
+//            in index order, so ties go to the lowest indices.  A token's output
+//            slot is its rank base + its rank by index among the block's tokens
+//            of equal distance.  From the candidate list (when it did not
+//            overflow): the listed tokens with D <= T are grouped by distance and
+//            ranked inside their group; otherwise two scans of all the block's
+//            distances find them (counts per warp, then an in-order emit, with a
+//            warp match over 32-entry chunks for the D < T tokens).  Either way
+//            the kept tokens end up in slot order, so both give the same bits.
+//            The kept K/V rows are prefetched into L2, gathered into registers
+//            (each half-warp keeps four K and four V rows in flight) and folded
+//            into an online-softmax state per half-warp; the states become one
+//            partial (m, l, o) per query head and block, which goes to the block
+//            that owns the head's merge.
 //   -- cluster barrier --
-//   merge    block 0 of the cluster combines the C partial states of each query
-//            head (peers' shared memory) into out and pads idx with -1.
-//   -- cluster barrier -- (no block leaves while a peer may still read it)
+//   merge    each block combines the C partial states of the query heads it owns
+//            (g mod C == its rank) into out; block 0 pads idx with -1.
 //
 // Every mbarrier wait is bounded: after kWaitLimit polls it sets
 // ADAMAS_DEVERR_TIMEOUT and goes on, so every thread still reaches every
@@ -56,7 +65,10 @@ namespace cg = cooperative_groups;
 
 constexpr int kWorkers = 512;                         // scoring / select / gather threads
 constexpr int kWorkerWarps = kWorkers / 32;
-constexpr int kThreads = kWorkers + 32;               // + the warp that issues the bulk copies
+constexpr int kCopyWarp = kWorkerWarps;               // issues the bulk copies of the code stream
+constexpr int kBoundWarp = kWorkerWarps + 1;          // keeps the candidate bounds of phase 1 tight
+constexpr int kThreads = kWorkers + 64;
+constexpr int kBoundRounds = 4096;                    // most bound updates of one step
 constexpr int kStageRows = 1024;                      // code rows per ring stage
 constexpr uint32_t kStageBytes = kStageRows * kCodeBytes;  // 32 KiB
 constexpr int kRowsPerThread = kStageRows / kWorkers;
@@ -65,10 +77,17 @@ constexpr int kMinStages = 2;
 constexpr int kMaxCluster = 16;
 constexpr int kHistStride = 388;                      // >= kBins, multiple of 4
 constexpr int kPartial = 132;                         // m, l, pad, pad, o[128]
-constexpr int kScratch = 256;                         // candidate entries per warp per 256-position group
-constexpr int kMaxKept = 2048;                        // kept tokens listed per sweep
+constexpr int kListCap = 4096;                        // D < T tokens listed per round / grouped candidates
+constexpr int kKeptCap = 4096;                        // kept tokens per gather window
+constexpr int kGroupMax = 512;                        // largest equal-distance group ranked from the candidate list
+constexpr int kCandMaxTokens = 65535;                 // candidate-list positions are 16-bit
 constexpr int kGatherRows = 4;                        // K/V rows in flight per half-warp
+constexpr int kScanBatch = 4;                         // 32-group iterations of a distance scan loaded together
+constexpr int kGatherBatch = 2 * kWorkerWarps * kGatherRows;  // rows per gather batch of the block
+constexpr int kPushHistMax = 8;                       // C * G up to which histograms are pushed to peers
+constexpr uint32_t kPosMask = (1u << 23) - 1u;        // token offset within a block (list entries: d << 23 | t)
 constexpr uint32_t kWaitLimit = 1u << 20;             // mbarrier polls (about a second)
+constexpr int kNoBound = 0x7FFF;                      // candidate bound before the block has k_eff tokens
 
 struct DecodeParams {
   const uint16_t* q;
@@ -86,37 +105,49 @@ struct DecodeParams {
   int cluster;          // blocks per (b, kv head)
   int nstages;          // ring stages, kMinStages..kMaxStages
   int dstride;          // distances per query head and block (>= any block's tokens, multiple of 64)
+  int clist_cap;        // candidate-list entries per query head (0: no candidate list)
 };
 
 // Shared-memory carve-up (bytes), shared with the host.
-//   head:    q codes [G][8], q words + masks [G][16], histograms [G][kHistStride],
-//            rank bases [G][kHistStride], partial states [G][kPartial]
-//   ring:    nstages x 32 KiB; in phase 2 it holds the per-warp counts
-//            [kWorkerWarps][kHistStride] (later the half-warp softmax states),
-//            the candidate scratch [kWorkerWarps][kScratch] and the kept list
-//   dist:    [G][dstride] u16 when kept in shared memory
+//   head:  q codes [G][8] | q words + masks [G][16] | own histograms [G][kHistStride]
+//          | rank bases [G][kHistStride] | own exclusive prefix [G][kHistStride]
+//          | histogram table [C][G][kHistStride] (when C*G <= kPushHistMax)
+//          | partial-state table [ceil(G/C)*C][kPartial]
+//   ring:  nstages x 32 KiB; in phase 2: per-warp chunk counts [kWorkerWarps][kHistStride]
+//          (later the half-warp softmax states), carried counts / group cursors
+//          [kHistStride], D < T tokens or grouped candidates [kListCap], kept tokens [kKeptCap]
+//   dist:  [G][dstride] u16 when kept in shared memory
+//   clist: [G][clist_cap] u16 candidate positions
 struct DecodeSmem {
   static __host__ __device__ inline size_t align128(size_t x) { return (x + 127) / 128 * 128; }
+  static __host__ __device__ inline bool push_hist(int G, int C) { return G * C <= kPushHistMax; }
+  static __host__ __device__ inline int owned(int G, int C) { return (G + C - 1) / C; }
   static __host__ __device__ inline size_t qcodes(int G) { return align128((size_t)G * kCodeWords * 4); }
   static __host__ __device__ inline size_t qconst(int G) { return align128((size_t)G * 2 * kCodeWords * 4); }
   static __host__ __device__ inline size_t hist(int G) { return align128((size_t)G * kHistStride * 4); }
-  static __host__ __device__ inline size_t partial(int G) { return align128((size_t)G * kPartial * 4); }
-  static __host__ __device__ inline size_t head(int G) {
-    return qcodes(G) + qconst(G) + 2 * hist(G) + partial(G);
+  static __host__ __device__ inline size_t htab(int G, int C) {
+    return push_hist(G, C) ? align128((size_t)C * G * kHistStride * 4) : 0;
+  }
+  static __host__ __device__ inline size_t ptab(int G, int C) {
+    return align128((size_t)owned(G, C) * C * kPartial * 4);
+  }
+  static __host__ __device__ inline size_t head(int G, int C) {
+    return qcodes(G) + qconst(G) + 3 * hist(G) + htab(G, C) + ptab(G, C);
   }
   static __host__ __device__ inline size_t ring(int nstages) { return (size_t)nstages * kStageBytes; }
   static constexpr __host__ __device__ size_t cnt() { return (size_t)kWorkerWarps * kHistStride * 4; }
-  static constexpr __host__ __device__ size_t scratch() { return (size_t)kWorkerWarps * kScratch * 4; }
+  static constexpr __host__ __device__ size_t carry() { return (size_t)kHistStride * 4; }
   static constexpr __host__ __device__ size_t state() { return (size_t)2 * kWorkerWarps * kPartial * 4; }
   static __host__ __device__ inline size_t dist(int G, int dstride, bool in_smem) {
     return in_smem ? align128((size_t)G * dstride * 2) : 0;
   }
-  static __host__ __device__ inline size_t total(int G, int nstages, int dstride, bool in_smem) {
-    return head(G) + ring(nstages) + dist(G, dstride, in_smem);
+  static __host__ __device__ inline size_t clist(int G, int cap) { return align128((size_t)G * cap * 2); }
+  static __host__ __device__ inline size_t total(int G, int C, int nstages, int dstride, bool in_smem, int cap) {
+    return head(G, C) + ring(nstages) + dist(G, dstride, in_smem) + clist(G, cap);
   }
 };
-static_assert(DecodeSmem::cnt() >= DecodeSmem::state(), "softmax states overlay the per-warp counts");
-static_assert(DecodeSmem::cnt() + DecodeSmem::scratch() + kMaxKept * 4 <= kMinStages * kStageBytes,
+static_assert(DecodeSmem::cnt() >= DecodeSmem::state(), "softmax states overlay the chunk counts");
+static_assert(DecodeSmem::cnt() + DecodeSmem::carry() + (kListCap + kKeptCap) * 4 <= kMinStages * kStageBytes,
               "phase-2 arrays fit in the smallest ring");
 
 // ------------------------------------------------------------------ block helpers
@@ -127,69 +158,184 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
-// Exclusive scan of one int64 per worker thread; returns the prefix and writes the
-// total to *total.  Uses sm_tmp[kWorkerWarps + 1].
-__device__ __forceinline__ int64_t worker_exclusive_scan(int64_t v, int64_t* sm_tmp, int64_t* total) {
+// Exclusive scan of one int64 per worker thread; returns the prefix.  Uses sm_tmp[kWorkerWarps].
+__device__ __forceinline__ long long worker_exclusive_scan(long long v, long long* sm_tmp) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int64_t x = v;
+  long long x = v;
 #pragma unroll
   for (int o = 1; o < 32; o *= 2) {
-    const int64_t y = __shfl_up_sync(0xffffffffu, x, o);
+    const long long y = __shfl_up_sync(0xffffffffu, x, o);
     if (lane >= o) x += y;
   }
   if (lane == 31) sm_tmp[warp] = x;
   worker_sync();
-  if (warp == 0) {
-    int64_t w = lane < kWorkerWarps ? sm_tmp[lane] : 0;
+  long long before = 0;
 #pragma unroll
-    for (int o = 1; o < 32; o *= 2) {
-      const int64_t y = __shfl_up_sync(0xffffffffu, w, o);
-      if (lane >= o) w += y;
-    }
-    if (lane < kWorkerWarps) sm_tmp[lane] = w;  // inclusive warp totals
-    if (lane == kWorkerWarps - 1) sm_tmp[kWorkerWarps] = w;
+  for (int w = 0; w < kWorkerWarps; ++w) before += w < warp ? sm_tmp[w] : 0;
+  worker_sync();
+  return before + x - v;
+}
+
+// Inclusive warp scan.
+__device__ __forceinline__ int warp_inclusive_scan(int x, int lane) {
+#pragma unroll
+  for (int o = 1; o < 32; o *= 2) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
   }
-  worker_sync();
-  const int64_t before = warp > 0 ? sm_tmp[warp - 1] : 0;
-  const int64_t res = before + x - v;
-  *total = sm_tmp[kWorkerWarps];
-  worker_sync();
-  return res;
+  return x;
 }
 
-// Distances of eight consecutive positions 8*grp .. 8*grp+7 (0xFFFF where grp is
-// past the warp's slice).
-__device__ __forceinline__ void load_dist8(const uint16_t* drow, int grp, bool in, uint32_t (&d)[8]) {
-  uint4 v = make_uint4(0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu);
-  if (in) v = *reinterpret_cast<const uint4*>(drow + (size_t)grp * 8);
-  d[0] = v.x & 0xFFFFu; d[1] = v.x >> 16; d[2] = v.y & 0xFFFFu; d[3] = v.y >> 16;
-  d[4] = v.z & 0xFFFFu; d[5] = v.z >> 16; d[6] = v.w & 0xFFFFu; d[7] = v.w >> 16;
-}
-
-// One K/V row (16 bytes of each per lane of a half-warp) folded into the
-// half-warp's online-softmax state.  Every lane of the warp calls it (the dot
-// product is reduced with shuffles inside the half-warp); `valid` is uniform
-// within a half-warp.
-__device__ __forceinline__ void softmax_fold(const float (&qf)[8], uint4 kr, uint4 vr, bool valid, float& m_run,
-                                             float& l_run, float (&o)[8]) {
-  float sc = 0.0f;
-  if (valid)
-    sc = qf[0] * bf16_lo(kr.x) + qf[1] * bf16_hi(kr.x) + qf[2] * bf16_lo(kr.y) + qf[3] * bf16_hi(kr.y) +
-         qf[4] * bf16_lo(kr.z) + qf[5] * bf16_hi(kr.z) + qf[6] * bf16_lo(kr.w) + qf[7] * bf16_hi(kr.w);
-  sc += __shfl_xor_sync(0xffffffffu, sc, 8);
-  sc += __shfl_xor_sync(0xffffffffu, sc, 4);
-  sc += __shfl_xor_sync(0xffffffffu, sc, 2);
-  sc += __shfl_xor_sync(0xffffffffu, sc, 1);
-  if (!valid) return;
-  const float m_new = fmaxf(m_run, sc);
-  const float corr = exp2f(m_run - m_new);
-  const float pr = exp2f(sc - m_new);
-  l_run = l_run * corr + pr;
-  const float vv[8] = {bf16_lo(vr.x), bf16_hi(vr.x), bf16_lo(vr.y), bf16_hi(vr.y),
-                       bf16_lo(vr.z), bf16_hi(vr.z), bf16_lo(vr.w), bf16_hi(vr.w)};
+// Smallest distance B with at least k tokens of the cluster's head at or below
+// it, from histograms that their blocks may still be adding to (any snapshot of
+// the counts gives a valid B, as every count read is of real tokens); -1 while
+// fewer than k tokens are counted.  Whole warp.  `hist` is this block's
+// histogram; with peers, the same histogram of every block of the cluster is
+// read (relaxed cluster-scope loads, all of a block's in flight together).
+__device__ __forceinline__ int kth_bound(const uint32_t* hist, int C, bool peers, int rank, int k, int lane) {
+  constexpr int kPer = (kBins + 31) / 32;
+  const uint32_t a0 = smem_addr(hist) + (uint32_t)(lane * kPer) * 4u;
+  int cnt[kPer];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) o[e] = o[e] * corr + pr * vv[e];
-  m_run = m_new;
+  for (int i = 0; i < kPer; ++i) cnt[i] = 0;
+  for (int r = 0; r < (peers ? C : 1); ++r) {
+    const uint32_t a = mapa_shared(a0, peers ? r : rank);
+    uint32_t v[kPer];
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) v[i] = lane * kPer + i < kBins ? ld_relaxed_cluster(a + 4u * i) : 0u;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) cnt[i] += (int)v[i];
+  }
+  int s = 0;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) s += cnt[i];
+  const int incl = warp_inclusive_scan(s, lane);
+  const uint32_t crossed = __ballot_sync(0xffffffffu, incl >= k);
+  if (crossed == 0u) return -1;
+  const int L = __ffs((int)crossed) - 1;
+  int res = 0, run = incl - s;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    run += cnt[i];
+    if (run >= k && res == 0 && lane == L) res = lane * kPer + i + 1;
+  }
+  return __shfl_sync(0xffffffffu, res, L) - 1;
+}
+
+// Eight consecutive distances 8*grp .. 8*grp+7 as four words of u16 pairs (element
+// 2j in the low half of word j); SMEM: the row is in shared memory.
+template <bool SMEM>
+__device__ __forceinline__ uint4 load_dist8(const uint16_t* drow, int grp) {
+  if constexpr (SMEM) return lds128(smem_addr(drow + (size_t)grp * 8));
+  else return *reinterpret_cast<const uint4*>(drow + (size_t)grp * 8);
+}
+
+template <bool SMEM>
+__device__ __forceinline__ uint32_t load_dist1(const uint16_t* drow, int pos) {
+  if constexpr (SMEM) {
+    uint16_t v;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(smem_addr(drow + pos)) : "memory");
+    return v;
+  } else {
+    return drow[pos];
+  }
+}
+
+constexpr uint32_t kHalfTops = 0x80008000u;
+
+// Whether any of the eight distances is <= T (t1x2 = (T+1) in both halves).  With
+// distances below 2^15 (0xFFFF pads a row), (x | 0x8000) - (T+1) keeps bit 15 of its
+// half exactly when x > T, and no half borrows from the other.
+__device__ __forceinline__ bool any_le(const uint4 v, uint32_t t1x2) {
+  const uint32_t a = ((v.x | kHalfTops) - t1x2) & ((v.y | kHalfTops) - t1x2) & ((v.z | kHalfTops) - t1x2) &
+                     ((v.w | kHalfTops) - t1x2);
+  return (a & kHalfTops) != kHalfTops;
+}
+
+// Bit e of lt (eq) set when distance e of the eight is < T (== T); tx2 = T in both
+// halves, t1x2 = T+1 in both halves.
+__device__ __forceinline__ void cand_bits(const uint4 v, uint32_t tx2, uint32_t t1x2, uint32_t& lt, uint32_t& eq) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  lt = 0u;
+  eq = 0u;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t ge = (w[j] | kHalfTops) - tx2;   // tops: x >= T
+    const uint32_t gt = (w[j] | kHalfTops) - t1x2;  // tops: x > T
+    const uint32_t l = ~ge & kHalfTops, e = ge & ~gt & kHalfTops;
+    lt |= ((l >> 15) & 1u) << (2 * j) | (l >> 31) << (2 * j + 1);
+    eq |= ((e >> 15) & 1u) << (2 * j) | (e >> 31) << (2 * j + 1);
+  }
+}
+
+// A batch of kGatherRows K/V rows (16 bytes of each per lane of a half-warp) folded
+// into the half-warp's online-softmax state: the scores first (reduced with
+// shuffles inside the half-warp; every lane of the warp takes part), then one
+// rescale for the batch.  valid[j] is uniform within a half-warp.
+__device__ __forceinline__ void softmax_fold(const float (&qf)[8], const uint4 (&kr)[kGatherRows],
+                                             const uint4 (&vr)[kGatherRows], const bool (&valid)[kGatherRows],
+                                             float& m_run, float& l_run, float (&o)[8]) {
+  float sc[kGatherRows];
+#pragma unroll
+  for (int j = 0; j < kGatherRows; ++j) {
+    const uint4 k = kr[j];
+    sc[j] = qf[0] * bf16_lo(k.x) + qf[1] * bf16_hi(k.x) + qf[2] * bf16_lo(k.y) + qf[3] * bf16_hi(k.y) +
+            qf[4] * bf16_lo(k.z) + qf[5] * bf16_hi(k.z) + qf[6] * bf16_lo(k.w) + qf[7] * bf16_hi(k.w);
+  }
+#pragma unroll
+  for (int off = 8; off > 0; off /= 2)
+#pragma unroll
+    for (int j = 0; j < kGatherRows; ++j) sc[j] += __shfl_xor_sync(0xffffffffu, sc[j], off);
+  bool any = false;
+  float mx = m_run;
+#pragma unroll
+  for (int j = 0; j < kGatherRows; ++j)
+    if (valid[j]) {
+      any = true;
+      mx = fmaxf(mx, sc[j]);
+    }
+  if (!any) return;
+  const float corr = exp2f(m_run - mx);  // 0 while the state is empty (m_run = -inf)
+  l_run *= corr;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) o[e] *= corr;
+#pragma unroll
+  for (int j = 0; j < kGatherRows; ++j)
+    if (valid[j]) {
+      const float pr = exp2f(sc[j] - mx);
+      l_run += pr;
+      const uint4 v = vr[j];
+      o[0] += pr * bf16_lo(v.x); o[1] += pr * bf16_hi(v.x); o[2] += pr * bf16_lo(v.y); o[3] += pr * bf16_hi(v.y);
+      o[4] += pr * bf16_lo(v.z); o[5] += pr * bf16_hi(v.z); o[6] += pr * bf16_lo(v.w); o[7] += pr * bf16_hi(v.w);
+    }
+  m_run = mx;
+}
+
+// K/V rows of kept entries rb + 32 j + (half-warp parity), j < kGatherRows, into
+// registers; `kept` holds token offsets within the block.
+__device__ __forceinline__ void gather_issue(const int32_t* kept, int rb, int n, int hw, int hl, const uint16_t* K,
+                                             const uint16_t* V, int64_t row0, uint4 (&kr)[kGatherRows],
+                                             uint4 (&vr)[kGatherRows]) {
+#pragma unroll
+  for (int j = 0; j < kGatherRows; ++j) {
+    const int row = rb + 2 * kWorkerWarps * j + (hw & 1);
+    kr[j] = make_uint4(0u, 0u, 0u, 0u);
+    vr[j] = kr[j];
+    if (row < n) {
+      const int64_t t = row0 + (int64_t)lds32(smem_addr(kept + row));
+      kr[j] = __ldcg(reinterpret_cast<const uint4*>(K + t * kDim) + hl);
+      vr[j] = __ldcg(reinterpret_cast<const uint4*>(V + t * kDim) + hl);
+    }
+  }
+}
+
+__device__ __forceinline__ void gather_fold(int rb, int n, int hw, const float (&qf)[8], const uint4 (&kr)[kGatherRows],
+                                            const uint4 (&vr)[kGatherRows], float& m_run, float& l_run,
+                                            float (&o)[8]) {
+  bool valid[kGatherRows];
+#pragma unroll
+  for (int j = 0; j < kGatherRows; ++j) valid[j] = rb + 2 * kWorkerWarps * j + (hw & 1) < n;
+  softmax_fold(qf, kr, vr, valid, m_run, l_run, o);
 }
 
 // ------------------------------------------------------------------ the kernel
@@ -200,11 +346,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const DecodePa
   __shared__ __align__(8) uint64_t sm_full[kMaxStages];
   __shared__ __align__(8) uint64_t sm_empty[kMaxStages];
   __shared__ int sm_T[kMaxGroup];
-  __shared__ int sm_kept_total;
-  __shared__ int sm_wlt[kWorkerWarps];    // per warp: candidates with D < T
-  __shared__ int sm_weq[kWorkerWarps];    // per warp: candidates with D == T
-  __shared__ int sm_wkept[kWorkerWarps];  // per warp: first position of its kept tokens in the list
-  __shared__ int64_t sm_scan[kWorkerWarps + 1];
+  __shared__ int sm_bound[kMaxGroup];   // candidate bound per query head (phase 1)
+  __shared__ int sm_scored;             // a worker warp has scored all its rows
+  __shared__ int sm_ncand[kMaxGroup][kWorkerWarps];  // candidates listed per query head and warp (may exceed the capacity)
+  __shared__ int sm_wlt[kWorkerWarps];  // per warp: candidates with D < T
+  __shared__ int sm_weq[kWorkerWarps];  // per warp: candidates with D == T
+  __shared__ int sm_wmax[kWorkerWarps];
+  __shared__ long long sm_tmp[kWorkerWarps];
 
   cg::cluster_group cluster = cg::this_cluster();
   const int C = p.cluster;
@@ -214,22 +362,34 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const DecodePa
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const bool worker = warp < kWorkerWarps;
   const uint32_t lt = (1u << lane) - 1u;
+  const bool push_hist = DecodeSmem::push_hist(G, C);
+  const int ccap = p.clist_cap;              // per query head: kWorkerWarps lists of wcap entries
+  const int wcap = ccap / kWorkerWarps;
+  const bool use_cand = ccap > 0;
 
   unsigned char* cur = smem;
-  uint32_t* sm_q = reinterpret_cast<uint32_t*>(cur);      cur += DecodeSmem::qcodes(G);   // [G][8]
-  uint32_t* sm_qc = reinterpret_cast<uint32_t*>(cur);     cur += DecodeSmem::qconst(G);   // [G][q 8 | m 8]
-  uint32_t* sm_hist = reinterpret_cast<uint32_t*>(cur);   cur += DecodeSmem::hist(G);     // [G][kHistStride]
-  uint32_t* sm_rank = reinterpret_cast<uint32_t*>(cur);   cur += DecodeSmem::hist(G);     // [G][kHistStride]
-  float* sm_part = reinterpret_cast<float*>(cur);         cur += DecodeSmem::partial(G);  // [G][kPartial]
+  uint32_t* sm_q = reinterpret_cast<uint32_t*>(cur);      cur += DecodeSmem::qcodes(G);    // [G][8]
+  uint32_t* sm_qc = reinterpret_cast<uint32_t*>(cur);     cur += DecodeSmem::qconst(G);    // [G][q 8 | m 8]
+  uint32_t* sm_hist = reinterpret_cast<uint32_t*>(cur);   cur += DecodeSmem::hist(G);      // [G][kHistStride]
+  uint32_t* sm_rank = reinterpret_cast<uint32_t*>(cur);   cur += DecodeSmem::hist(G);      // [G][kHistStride]
+  uint32_t* sm_lpre = reinterpret_cast<uint32_t*>(cur);   cur += DecodeSmem::hist(G);      // [G][kHistStride]
+  uint32_t* sm_htab = reinterpret_cast<uint32_t*>(cur);   cur += DecodeSmem::htab(G, C);   // [C][G][kHistStride]
+  float* sm_ptab = reinterpret_cast<float*>(cur);         cur += DecodeSmem::ptab(G, C);   // [owned*C][kPartial]
   unsigned char* ring = cur;                              cur += DecodeSmem::ring(p.nstages);
   uint16_t* dist;
-  if constexpr (SMEM_D) dist = reinterpret_cast<uint16_t*>(cur);
-  else dist = p.dglobal + (size_t)blockIdx.x * G * p.dstride;
+  if constexpr (SMEM_D) {
+    dist = reinterpret_cast<uint16_t*>(cur);
+    cur += DecodeSmem::dist(G, p.dstride, true);
+  } else {
+    dist = p.dglobal + (size_t)blockIdx.x * G * p.dstride;
+  }
+  uint16_t* sm_cand = reinterpret_cast<uint16_t*>(cur);  // [G][kWorkerWarps][wcap]
   // phase-2 arrays over the ring
-  uint32_t* sm_cnt = reinterpret_cast<uint32_t*>(ring);                                    // [kWorkerWarps][kHistStride]
-  float* sm_state = reinterpret_cast<float*>(ring);                                        // [2*kWorkerWarps][kPartial]
-  uint32_t* sm_scratch = reinterpret_cast<uint32_t*>(ring + DecodeSmem::cnt());            // [kWorkerWarps][kScratch]
-  int32_t* sm_kept = reinterpret_cast<int32_t*>(ring + DecodeSmem::cnt() + DecodeSmem::scratch());  // [kMaxKept]
+  uint32_t* sm_cnt = reinterpret_cast<uint32_t*>(ring);                          // [kWorkerWarps][kHistStride]
+  float* sm_state = reinterpret_cast<float*>(ring);                              // [2*kWorkerWarps][kPartial]
+  uint32_t* sm_carry = reinterpret_cast<uint32_t*>(ring + DecodeSmem::cnt());    // [kHistStride]
+  int32_t* sm_list = reinterpret_cast<int32_t*>(ring + DecodeSmem::cnt() + DecodeSmem::carry());  // [kListCap]
+  int32_t* sm_kept = sm_list + kListCap;                                         // [kKeptCap]
 
   // ---- the head's length and this block's tokens
   int64_t len_b = p.seq_lens[b];
@@ -252,10 +412,37 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const DecodePa
     fence_mbar_init();
   }
   for (int i = tid; i < G * kHistStride; i += kThreads) sm_hist[i] = 0u;
+  if (tid < kMaxGroup) {
+    sm_T[tid] = kBins - 1;  // always overwritten when the histograms are consistent
+    sm_bound[tid] = kNoBound;
+  }
+  if (tid == 0) sm_scored = 0;
   __syncthreads();
+  // Peers read this block's histograms during phase 1 (candidate bounds): every
+  // thread arrives on a cluster barrier once the histograms are cleared and waits
+  // on it before it (or a peer, in turn) can look at another block -- after the
+  // first stage, long after every block has arrived.
+  cluster_arrive();
+  bool waited = false;
 
   // ================================================================ phase 1
-  if (!worker) {
+  if (warp == kBoundWarp) {
+    // Recompute the candidate bounds from the whole cluster's histograms until the
+    // stream is scored; the workers only read them.
+    cluster_wait();
+    waited = true;
+    if (use_cand && nst > 0)
+      for (int it = 0; it < kBoundRounds; ++it) {
+        if (*(volatile int*)&sm_scored) break;
+#pragma unroll 1
+        for (int g = 0; g < G; ++g) {
+          const int bnd = kth_bound(sm_hist + g * kHistStride, C, true, rank, keff, lane);
+          if (bnd >= 0 && lane == 0) atomicMin(&sm_bound[g], bnd);
+        }
+        __syncwarp();
+        __nanosleep(500);
+      }
+  } else if (!worker) {
     if (lane == 0) {
       const unsigned char* src = p.codes + (kv_base + t0) * kCodeBytes;
       for (int i = 0; i < nst; ++i) {
@@ -289,21 +476,31 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const DecodePa
           rm[g][w] = sm_qc[g * 2 * kCodeWords + kCodeWords + w];
         }
     }
+    int ncand[G];  // this warp's listed candidates per query head (uniform in the warp)
+#pragma unroll
+    for (int g = 0; g < G; ++g) ncand[g] = 0;
     for (int i = 0; i < nst; ++i) {
       const int buf = i % NS;
       if (!mbar_wait(&sm_full[buf], (uint32_t)(i / NS) & 1u, kWaitLimit)) atomicOr(p.err, kErrTimeout);
       const int rows = min(kStageRows, seg_len - i * kStageRows);
       const unsigned char* st = ring + (size_t)buf * kStageBytes;
+      int bound[G];
+#pragma unroll
+      for (int g = 0; g < G; ++g) bound[g] = use_cand ? *(volatile int*)&sm_bound[g] : -1;
+      int dg[kRowsPerThread][G];  // kNoBound + 1 for rows past the stage's end
 #pragma unroll
       for (int j = 0; j < kRowsPerThread; ++j) {
         const int r = j * kWorkers + tid;
+        const int t = i * kStageRows + r;
+#pragma unroll
+        for (int g = 0; g < G; ++g) dg[j][g] = kNoBound + 1;
         if (r < rows) {
-          const uint4 x0 = *reinterpret_cast<const uint4*>(st + (size_t)r * kCodeBytes);
-          const uint4 x1 = *reinterpret_cast<const uint4*>(st + (size_t)r * kCodeBytes + 16);
+          const uint32_t ra = smem_addr(st + (size_t)r * kCodeBytes);
+          const uint4 x0 = lds128(ra);
+          const uint4 x1 = lds128(ra + 16);
           const uint32_t k[kCodeWords] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
           uint32_t k1[kCodeWords];
           key_shift(k, k1);
-          const int t = i * kStageRows + r;
 #pragma unroll
           for (int g = 0; g < G; ++g) {
             int d;
@@ -319,50 +516,87 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const DecodePa
               mg[4] = m1.x; mg[5] = m1.y; mg[6] = m1.z; mg[7] = m1.w;
               d = l1_distance(k, k1, qg, mg);
             }
-            dist[(size_t)g * p.dstride + t] = (uint16_t)d;
+            dg[j][g] = d;
+            if constexpr (SMEM_D) sts16(smem_addr(dist + (size_t)g * p.dstride + t), (uint16_t)d);
+            else dist[(size_t)g * p.dstride + t] = (uint16_t)d;
             atomicAdd(&sm_hist[g * kHistStride + d], 1u);
           }
         }
       }
+      if (use_cand) {
+#pragma unroll
+        for (int j = 0; j < kRowsPerThread; ++j)
+#pragma unroll
+          for (int g = 0; g < G; ++g) {  // list the row if it can still be selected
+            const bool pred = dg[j][g] <= bound[g];
+            const uint32_t m = __ballot_sync(0xffffffffu, pred);
+            const int at = ncand[g] + __popc(m & lt);
+            if (pred && at < wcap)
+              sm_cand[(size_t)g * ccap + warp * wcap + at] = (uint16_t)(i * kStageRows + j * kWorkers + tid);
+            ncand[g] += __popc(m);
+          }
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm_empty[buf]);
     }
+    if (lane == 0) *(volatile int*)&sm_scored = 1;
+    if (lane == 0)
+#pragma unroll
+      for (int g = 0; g < G; ++g) sm_ncand[g][warp] = ncand[g];
+    if (push_hist && keff > 0) {  // own histograms into every block's table (row `rank`)
+      worker_sync();
+      for (int r = 0; r < C; ++r) {
+        uint32_t* tab = cluster.map_shared_rank(sm_htab, r) + (size_t)rank * G * kHistStride;
+        for (int i = tid; i < G * kHistStride; i += kWorkers) tab[i] = sm_hist[i];
+      }
+    }
   }
+  if (!waited) cluster_wait();
   __syncthreads();
   cluster.sync();  // every block's histograms are complete and visible to the cluster
 
   // ================================================================ phase 2
   if (worker && keff > 0) {
-    // ---- thresholds and rank bases of every query head (histograms of the whole cluster)
-    if (tid < G) sm_T[tid] = kBins - 1;  // always overwritten when the histograms are consistent
-    worker_sync();
+    // ---- the tail of the last 8-position group of every distance row reads as "far"
+    if (tid < G)
+      for (int pos = seg_len; pos < ((seg_len + 7) & ~7); ++pos) {
+        if constexpr (SMEM_D) sts16(smem_addr(dist + (size_t)tid * p.dstride + pos), 0xFFFFu);
+        else dist[(size_t)tid * p.dstride + pos] = 0xFFFFu;
+      }
+    // ---- thresholds, rank bases and own prefixes of every query head
     for (int g = 0; g < G; ++g) {
       const int d = tid;  // bins 0..kBins-1 on the first kBins threads
-      int64_t H = 0, P = 0;
+      long long H = 0, P = 0, own = 0;
       if (d < kBins) {
         uint32_t v[kMaxCluster];
 #pragma unroll
-        for (int r = 0; r < kMaxCluster; ++r)
-          v[r] = r < C ? cluster.map_shared_rank(sm_hist, r)[g * kHistStride + d] : 0u;
+        for (int r = 0; r < kMaxCluster; ++r) {
+          v[r] = 0u;
+          if (r < C)
+            v[r] = push_hist ? sm_htab[((size_t)r * G + g) * kHistStride + d]
+                             : cluster.map_shared_rank(sm_hist, r)[g * kHistStride + d];
+        }
 #pragma unroll
         for (int r = 0; r < kMaxCluster; ++r) {
           H += v[r];
           if (r < rank) P += v[r];
         }
+        own = sm_hist[g * kHistStride + d];
       }
-      int64_t tot;
-      const int64_t base = worker_exclusive_scan(H, sm_scan, &tot);
+      // both prefixes in one scan: totals of the head in the high word, own counts in the low one
+      const long long pre = worker_exclusive_scan(H << 32 | own, sm_tmp);
+      const int base = (int)(pre >> 32);
       if (d < kBins) {
         if (base < keff && base + H >= keff) sm_T[g] = d;
         sm_rank[g * kHistStride + d] = (uint32_t)(base + P);
+        sm_lpre[g * kHistStride + d] = (uint32_t)(pre & 0xFFFFFFFFll);
       }
     }
     worker_sync();
 
     const int hw = tid >> 4, hl = tid & 15;  // 32 half-warps
     const float kScoreScale = 0.08838834764831845f * 1.4426950408889634f;  // log2(e)/sqrt(128)
-    uint32_t* scr = sm_scratch + warp * kScratch;
-    // warp slices over 8-position groups of the block's distances
+    // warp slices over 8-position groups of the block's distances (full scans)
     const int ngrp = (seg_len + 7) >> 3;
     const int gpw = (ngrp + kWorkerWarps - 1) / kWorkerWarps;
     const int wg0 = min(ngrp, warp * gpw), wg1 = min(ngrp, (warp + 1) * gpw);
@@ -372,149 +606,253 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const DecodePa
       int32_t* idx_h = p.idx + hq * p.budget;
       const uint16_t* drow = dist + (size_t)g * p.dstride;
       const uint32_t* rank_g = sm_rank + g * kHistStride;
+      const uint32_t* lpre_g = sm_lpre + g * kHistStride;
+      const uint32_t* hist_g = sm_hist + g * kHistStride;
       const uint32_t T = (uint32_t)sm_T[g];
+      const int tie_base = (int)rank_g[T];              // output slot of this block's first tie
+      const int tie_quota = max(0, keff - tie_base);    // ties this block keeps (its first ones)
+      const int n_lt = (int)lpre_g[T];                  // tokens of the block with D < T
+      const int n_eq = (int)hist_g[T];                  // ties of the block
+      const int n_kept = n_lt + min(tie_quota, n_eq);   // kept tokens, in slot order at [0, n_kept)
+      const uint4 qraw = *reinterpret_cast<const uint4*>(p.q + hq * kDim + 8 * hl);
+
+      // largest group of equal distances <= T, and whether the candidate list serves
+      {
+        const int v = (tid <= (int)T) ? (int)hist_g[tid] : 0;
+        const int m = __reduce_max_sync(0xffffffffu, v);
+        if (lane == 0) sm_wmax[warp] = m;
+      }
+      for (int i = tid; i < kHistStride; i += kWorkers) sm_carry[i] = 0u;
+      worker_sync();
+      int gmax = 0, cmax = 0;
+#pragma unroll
+      for (int w = 0; w < kWorkerWarps; ++w) {
+        gmax = max(gmax, sm_wmax[w]);
+        cmax = max(cmax, sm_ncand[g][w]);
+      }
+      bool from_list = use_cand && cmax <= wcap && n_lt + n_eq <= kListCap && n_kept <= kKeptCap &&
+                       gmax <= kGroupMax;
 
       float qf[8];
-      {
-        const uint4 qr = *reinterpret_cast<const uint4*>(p.q + hq * kDim + 8 * hl);
-        qf[0] = bf16_lo(qr.x) * kScoreScale; qf[1] = bf16_hi(qr.x) * kScoreScale;
-        qf[2] = bf16_lo(qr.y) * kScoreScale; qf[3] = bf16_hi(qr.y) * kScoreScale;
-        qf[4] = bf16_lo(qr.z) * kScoreScale; qf[5] = bf16_hi(qr.z) * kScoreScale;
-        qf[6] = bf16_lo(qr.w) * kScoreScale; qf[7] = bf16_hi(qr.w) * kScoreScale;
-      }
       float m_run = -INFINITY, l_run = 0.0f, o[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) o[e] = 0.0f;
 
-      // sweeps of at most kMaxKept kept tokens (one sweep unless the block keeps more)
-      for (int c0 = 0;; c0 += kMaxKept) {
-        for (int i = tid; i < kWorkerWarps * kHistStride; i += kWorkers) sm_cnt[i] = 0u;
+      // gather of the kept tokens [0, n) of one window into the softmax state
+      auto gather = [&](int n, bool prefetch) {
+        for (int i = tid; prefetch && i < 4 * n; i += kWorkers) {  // every kept row on its way into L2
+          const int64_t t = kv_base + t0 + (int64_t)lds32(smem_addr(sm_kept + (i >> 2)));
+          prefetch_l2((i & 2 ? p.V : p.K) + t * kDim + (i & 1) * 64);
+        }
+        for (int rb = 2 * warp; rb < n; rb += kGatherBatch) {
+          uint4 kr[kGatherRows], vr[kGatherRows];
+          gather_issue(sm_kept, rb, n, hw, hl, p.K, p.V, kv_base + t0, kr, vr);
+          gather_fold(rb, n, hw, qf, kr, vr, m_run, l_run, o);
+        }
+      };
+
+      if (from_list) {
+        // ---- candidates with D <= T grouped by distance (group d at [lpre[d], lpre[d] + hist[d]))
+        const uint16_t* cand = sm_cand + (size_t)g * ccap + warp * wcap;  // this warp's phase-1 list
+        const int nw = sm_ncand[g][warp];
+        for (int x = lane; x < nw; x += 32) {
+          uint16_t tpos;
+          asm volatile("ld.shared.u16 %0, [%1];" : "=h"(tpos) : "r"(smem_addr(cand + x)) : "memory");
+          const uint32_t d = load_dist1<SMEM_D>(drow, tpos);
+          if (d <= T) {
+            const uint32_t c = atomicAdd(&sm_carry[d], 1u);
+            if (c >= hist_g[d]) continue;  // never with a complete list (checked below)
+            sm_list[lpre_g[d] + c] = (int32_t)(d << 23 | tpos);
+            const int64_t row = kv_base + t0 + tpos;  // the row is very likely kept: on its way into L2
+            prefetch_l2(p.K + row * kDim);
+            prefetch_l2(p.K + row * kDim + 64);
+            prefetch_l2(p.V + row * kDim);
+            prefetch_l2(p.V + row * kDim + 64);
+          }
+        }
         worker_sync();
-        // ---- pass 1: per-warp counts of the candidates (D <= T) per distance
-        int nlt = 0, neq = 0;
-        for (int gb = wg0; gb < wg1; gb += 32) {
-          const int grp = gb + lane;
-          uint32_t dv[8];
-          load_dist8(drow, grp, grp < wg1, dv);
+        // every group must be complete (each token with D <= T listed once), else the scans decide
+        if (tid == 0) sm_wmax[0] = 0;
+        worker_sync();
+        if (tid <= (int)T && sm_carry[tid] != hist_g[tid]) sm_wmax[0] = 1;
+        worker_sync();
+        from_list = sm_wmax[0] == 0;
+        worker_sync();
+      }
+      if (from_list) {
+        // ---- rank inside the group by index: slot, and the kept position lpre[d] + rank
+        const int nf = n_lt + n_eq;
+        for (int i = tid; i < nf; i += kWorkers) {
+          const uint32_t e = lds32(smem_addr(sm_list + i));
+          const uint32_t d = e >> 23, tpos = e & kPosMask;
+          const int gb = (int)lpre_g[d], gn = (int)hist_g[d];
+          int r = 0;
+          for (int q = gb; q < gb + gn; ++q) r += (lds32(smem_addr(sm_list + q)) & kPosMask) < tpos;
+          const int slot = (int)rank_g[d] + r;
+          if (slot < keff) {
+            idx_h[slot] = (int32_t)(t0 + tpos);
+            sm_kept[gb + r] = (int32_t)tpos;
+          }
+        }
+        worker_sync();
+        qf[0] = bf16_lo(qraw.x) * kScoreScale; qf[1] = bf16_hi(qraw.x) * kScoreScale;
+        qf[2] = bf16_lo(qraw.y) * kScoreScale; qf[3] = bf16_hi(qraw.y) * kScoreScale;
+        qf[4] = bf16_lo(qraw.z) * kScoreScale; qf[5] = bf16_hi(qraw.z) * kScoreScale;
+        qf[6] = bf16_lo(qraw.w) * kScoreScale; qf[7] = bf16_hi(qraw.w) * kScoreScale;
+        gather(n_kept, false);
+        worker_sync();
+      }
+      if (!from_list) {
+        // ---- count pass: candidates per warp
+        const uint32_t tx2 = T | T << 16, t1x2 = (T + 1) | (T + 1) << 16;
+        int c_lt = 0, c_eq = 0;
+        for (int gb0 = wg0; gb0 < wg1; gb0 += 32 * kScanBatch) {
+          uint4 v[kScanBatch];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int pos = grp * 8 + e;
-            if (dv[e] <= T && pos < seg_len) {
-              atomicAdd(&sm_cnt[warp * kHistStride + dv[e]], 1u);
-              nlt += dv[e] < T;
-              neq += dv[e] == T;
+          for (int it = 0; it < kScanBatch; ++it) {
+            const int grp = gb0 + 32 * it + lane;
+            v[it] = grp < wg1 ? load_dist8<SMEM_D>(drow, grp) : make_uint4(~0u, ~0u, ~0u, ~0u);
+          }
+#pragma unroll
+          for (int it = 0; it < kScanBatch; ++it)
+            if (any_le(v[it], t1x2)) {
+              uint32_t mlt, meq;
+              cand_bits(v[it], tx2, t1x2, mlt, meq);
+              c_lt += __popc(mlt);
+              c_eq += __popc(meq);
             }
-          }
         }
-#pragma unroll
-        for (int o2 = 16; o2 > 0; o2 /= 2) {
-          nlt += __shfl_xor_sync(0xffffffffu, nlt, o2);
-          neq += __shfl_xor_sync(0xffffffffu, neq, o2);
-        }
+        c_lt = __reduce_add_sync(0xffffffffu, c_lt);
+        c_eq = __reduce_add_sync(0xffffffffu, c_eq);
         if (lane == 0) {
-          sm_wlt[warp] = nlt;
-          sm_weq[warp] = neq;
+          sm_wlt[warp] = c_lt;
+          sm_weq[warp] = c_eq;
         }
         worker_sync();
-        for (int d = tid; d <= (int)T; d += kWorkers) {  // exclusive prefix over the warps, per distance
-          uint32_t run = 0;
-          for (int w = 0; w < kWorkerWarps; ++w) {
-            const uint32_t cw = sm_cnt[w * kHistStride + d];
-            sm_cnt[w * kHistStride + d] = run;
-            run += cw;
-          }
+        int lt_base = 0, eq_base = 0;
+#pragma unroll
+        for (int w = 0; w < kWorkerWarps; ++w) {
+          lt_base += w < warp ? sm_wlt[w] : 0;
+          eq_base += w < warp ? sm_weq[w] : 0;
         }
-        if (tid == 0) {  // kept tokens per warp: every D < T, and the ties at T within the quota
-          const int tie0 = (int)rank_g[T];
-          int ties_before = 0, kept_before = 0;
-          for (int w = 0; w < kWorkerWarps; ++w) {
-            const int ties = min(max(keff - (tie0 + ties_before), 0), sm_weq[w]);
-            sm_wkept[w] = kept_before;
-            kept_before += sm_wlt[w] + ties;
-            ties_before += sm_weq[w];
-          }
-          sm_kept_total = kept_before;
-        }
-        worker_sync();
-        const int kept_total = sm_kept_total;
-        // ---- pass 2: in index order, every candidate to its final slot
-        int kept_at = sm_wkept[warp];
-        for (int gb = wg0; gb < wg1; gb += 32) {
-          const int grp = gb + lane;
-          uint32_t dv[8];
-          load_dist8(drow, grp, grp < wg1, dv);
-          uint32_t mask = 0;
+        qf[0] = bf16_lo(qraw.x) * kScoreScale; qf[1] = bf16_hi(qraw.x) * kScoreScale;
+        qf[2] = bf16_lo(qraw.y) * kScoreScale; qf[3] = bf16_hi(qraw.y) * kScoreScale;
+        qf[4] = bf16_lo(qraw.z) * kScoreScale; qf[5] = bf16_hi(qraw.z) * kScoreScale;
+        qf[6] = bf16_lo(qraw.w) * kScoreScale; qf[7] = bf16_hi(qraw.w) * kScoreScale;
+
+        // windows of kKeptCap kept positions; per window, rounds of kListCap D < T tokens
+        for (int c0 = 0; c0 < n_kept; c0 += kKeptCap) {
+          const int n_win = min(kKeptCap, n_kept - c0);
+          for (int r0 = 0; r0 == 0 || r0 < n_lt; r0 += kListCap) {
+            const int n_round = max(0, min(kListCap, n_lt - r0));
+            // ---- emit pass: the round's D < T tokens to the list; ties (first round) to their slots
+            int lt_run = lt_base, eq_run = eq_base;
+            for (int gb0 = wg0; gb0 < wg1; gb0 += 32 * kScanBatch) {
+              uint4 v[kScanBatch];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int pos = grp * 8 + e;
-            if (dv[e] <= T && pos < seg_len) mask |= 1u << e;
-          }
-          const int cnum = __popc(mask);
-          if (__ballot_sync(0xffffffffu, cnum != 0) == 0u) continue;
-          int incl = cnum;
+              for (int it = 0; it < kScanBatch; ++it) {
+                const int grp = gb0 + 32 * it + lane;
+                v[it] = grp < wg1 ? load_dist8<SMEM_D>(drow, grp) : make_uint4(~0u, ~0u, ~0u, ~0u);
+              }
+              uint32_t mlt[kScanBatch], meq[kScanBatch];
+              int incl[kScanBatch];
+              bool mine = false;
 #pragma unroll
-          for (int o2 = 1; o2 < 32; o2 *= 2) {
-            const int y = __shfl_up_sync(0xffffffffu, incl, o2);
-            if (lane >= o2) incl += y;
-          }
-          const int total = __shfl_sync(0xffffffffu, incl, 31);
-          int at = incl - cnum;
+              for (int it = 0; it < kScanBatch; ++it) {
+                mlt[it] = 0u;
+                meq[it] = 0u;
+                if (any_le(v[it], t1x2)) cand_bits(v[it], tx2, t1x2, mlt[it], meq[it]);
+                incl[it] = __popc(mlt[it]) | __popc(meq[it]) << 16;
+                mine |= incl[it] != 0;
+              }
+              if (__ballot_sync(0xffffffffu, mine) == 0u) continue;
+              int own[kScanBatch];
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            if (mask & (1u << e)) scr[at++] = (uint32_t)(grp * 8 + e) << 9 | dv[e];
-          __syncwarp();
-          for (int k0 = 0; k0 < total; k0 += 32) {
-            const int k = k0 + lane;
-            const bool valid = k < total;
-            const uint32_t ent = valid ? scr[k] : 0u;
-            const uint32_t d = ent & 511u;
-            const uint32_t m = __ballot_sync(0xffffffffu, valid);
-            uint32_t peers = 0;
-            bool kept = false;
-            if (valid) {
-              peers = __match_any_sync(m, d);
-              const uint32_t slot = rank_g[d] + sm_cnt[warp * kHistStride + d] + __popc(peers & lt);
-              if (slot < (uint32_t)keff) {
-                kept = true;
-                if (c0 == 0) idx_h[slot] = (int32_t)(t0 + (int64_t)(ent >> 9));
+              for (int it = 0; it < kScanBatch; ++it) own[it] = incl[it];
+#pragma unroll
+              for (int off = 1; off < 32; off *= 2)
+#pragma unroll
+                for (int it = 0; it < kScanBatch; ++it) {
+                  const int y = __shfl_up_sync(0xffffffffu, incl[it], off);
+                  if (lane >= off) incl[it] += y;
+                }
+#pragma unroll
+              for (int it = 0; it < kScanBatch; ++it) {
+                const int tot = __shfl_sync(0xffffffffu, incl[it], 31);
+                if (own[it] != 0) {
+                  const int grp = gb0 + 32 * it + lane;
+                  int at_lt = lt_run + ((incl[it] - own[it]) & 0xFFFF);
+                  int at_eq = eq_run + ((incl[it] - own[it]) >> 16);
+                  const uint32_t w[4] = {v[it].x, v[it].y, v[it].z, v[it].w};
+#pragma unroll
+                  for (int e = 0; e < 8; ++e) {
+                    const uint32_t pos = (uint32_t)(grp * 8 + e);
+                    const uint32_t dval = (w[e >> 1] >> (16 * (e & 1))) & 0xFFFFu;
+                    if (mlt[it] & (1u << e)) {
+                      const int k = at_lt++ - r0;
+                      if (k >= 0 && k < n_round) sm_list[k] = (int32_t)(dval << 23 | pos);
+                    }
+                    if (r0 == 0 && (meq[it] & (1u << e))) {
+                      const int tie = at_eq++;
+                      if (tie < tie_quota) {
+                        if (c0 == 0) idx_h[tie_base + tie] = (int32_t)(t0 + pos);
+                        const int kp = n_lt + tie - c0;
+                        if (kp >= 0 && kp < n_win) sm_kept[kp] = (int32_t)pos;
+                      }
+                    }
+                  }
+                }
+                lt_run += tot & 0xFFFF;
+                eq_run += tot >> 16;
               }
             }
-            const uint32_t kb = __ballot_sync(0xffffffffu, kept);
-            const int pos_k = kept_at + __popc(kb & lt);
-            if (kept && pos_k >= c0 && pos_k < c0 + kMaxKept) sm_kept[pos_k - c0] = (int32_t)(ent >> 9);
-            kept_at += __popc(kb);
-            __syncwarp();
-            if (valid && (peers & lt) == 0u) sm_cnt[warp * kHistStride + d] += __popc(peers);
-            __syncwarp();
-          }
-        }
-        worker_sync();
-        // ---- gather the listed rows straight into registers; the trip count depends
-        // on the warp only, so both half-warps always reach the shuffles together
-        const int n_list = max(0, min(kMaxKept, kept_total - c0));
-        for (int rb = 2 * warp; rb < n_list; rb += 2 * kWorkerWarps * kGatherRows) {
-          uint4 kr[kGatherRows], vr[kGatherRows];
+            worker_sync();
+            // ---- slots of the round's D < T tokens: rank among equal distances by index
+            if (r0 == 0)
+              for (int i = tid; i < kHistStride; i += kWorkers) sm_carry[i] = 0u;
+            for (int i = tid; i < kWorkerWarps * kHistStride; i += kWorkers) sm_cnt[i] = 0u;
+            worker_sync();
+            for (int q0 = 0; q0 < n_round; q0 += kWorkers) {
+              const int i = q0 + tid;
+              const bool valid = i < n_round;
+              const uint32_t ent = valid ? lds32(smem_addr(sm_list + i)) : 0u;
+              const uint32_t d = ent >> 23;
+              const uint32_t m = __ballot_sync(0xffffffffu, valid);
+              uint32_t peers = 0u;
+              if (valid) {
+                peers = __match_any_sync(m, d);
+                if ((peers & lt) == 0u) sm_cnt[warp * kHistStride + d] = (uint32_t)__popc(peers);
+              }
+              worker_sync();
+              if (valid) {
+                const uint32_t ca = smem_addr(sm_cnt + d);
+                uint32_t before = lds32(smem_addr(sm_carry + d));
 #pragma unroll
-          for (int j = 0; j < kGatherRows; ++j) {
-            const int row = rb + 2 * kWorkerWarps * j + (hw & 1);
-            kr[j] = make_uint4(0u, 0u, 0u, 0u);
-            vr[j] = kr[j];
-            if (row < n_list) {
-              const int64_t t = t0 + sm_kept[row];
-              kr[j] = __ldcg(reinterpret_cast<const uint4*>(p.K + (kv_base + t) * kDim) + hl);
-              vr[j] = __ldcg(reinterpret_cast<const uint4*>(p.V + (kv_base + t) * kDim) + hl);
+                for (int w = 0; w < kWorkerWarps - 1; ++w)
+                  if (w < warp) before += lds32(ca + w * kHistStride * 4);
+                before += (uint32_t)__popc(peers & lt);  // rank of the token among the block's equal distances
+                const uint32_t tpos = ent & kPosMask;
+                if (c0 == 0 && rank_g[d] + before < (uint32_t)keff) idx_h[rank_g[d] + before] = (int32_t)(t0 + tpos);
+                const int kp = (int)(lpre_g[d] + before) - c0;
+                if (kp >= 0 && kp < n_win) sm_kept[kp] = (int32_t)tpos;
+              }
+              worker_sync();
+              for (int dd = tid; dd < kBins; dd += kWorkers) {  // counts carried to later entries
+                uint32_t s = 0u;
+                for (int w = 0; w < kWorkerWarps; ++w) {
+                  s += sm_cnt[w * kHistStride + dd];
+                  sm_cnt[w * kHistStride + dd] = 0u;
+                }
+                sm_carry[dd] += s;
+              }
+              worker_sync();
             }
           }
-#pragma unroll
-          for (int j = 0; j < kGatherRows; ++j) {
-            const int row = rb + 2 * kWorkerWarps * j + (hw & 1);
-            softmax_fold(qf, kr[j], vr[j], row < n_list, m_run, l_run, o);
-          }
+          gather(n_win, true);
+          worker_sync();
         }
-        worker_sync();
-        if (c0 + kMaxKept >= kept_total) break;
       }
-      // ---- half-warp states -> this block's partial state for the query head
+      // ---- half-warp states -> this block's partial state -> the head's owner
       {
         float* st = sm_state + hw * kPartial;
         if (hl == 0) { st[0] = m_run; st[1] = l_run; }
@@ -534,53 +872,45 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const DecodePa
             O += sk[4 + tid] * wgt;
           }
         }
-        sm_part[g * kPartial + 4 + tid] = O;
-        if (tid == 0) { sm_part[g * kPartial] = M; sm_part[g * kPartial + 1] = L; }
+        float* dst = cluster.map_shared_rank(sm_ptab, g % C) + ((size_t)(g / C) * C + rank) * kPartial;
+        dst[4 + tid] = O;
+        if (tid == 0) { dst[0] = M; dst[1] = L; }
       }
       worker_sync();
     }
   }
   __syncthreads();
-  cluster.sync();  // every block's partial states are complete
+  cluster.sync();  // every partial state is in its owner's table
 
-  // ================================================================ merge (block 0 of the cluster)
-  if (rank == 0 && worker) {
-    for (int i = tid; i < G * kDim; i += kWorkers) {
-      const int g = i / kDim, e = i - g * kDim;
+  // ================================================================ merge of the owned query heads
+  if (worker) {
+    for (int g = rank; g < G; g += C) {
       const int64_t hq = (int64_t)b * p.Hq + kvh * G + g;
-      float res = 0.0f;
-      if (keff > 0) {
-        float mv[kMaxCluster], lv[kMaxCluster], ov[kMaxCluster];
-#pragma unroll
-        for (int r = 0; r < kMaxCluster; ++r) {
-          mv[r] = -INFINITY; lv[r] = 0.0f; ov[r] = 0.0f;
-          if (r < C) {
-            const float* pr = cluster.map_shared_rank(sm_part, r) + g * kPartial;
-            mv[r] = pr[0]; lv[r] = pr[1]; ov[r] = pr[4 + e];
+      for (int e = tid; e < kDim; e += kWorkers) {
+        float res = 0.0f;
+        if (keff > 0) {
+          const float* tab = sm_ptab + (size_t)(g / C) * C * kPartial;
+          float M = -INFINITY;
+          for (int r = 0; r < C; ++r) M = fmaxf(M, tab[r * kPartial]);
+          float L = 0.0f, O = 0.0f;
+          for (int r = 0; r < C; ++r) {
+            const float mr = tab[r * kPartial];
+            if (mr == -INFINITY) continue;  // a block that kept no token of this head
+            const float wgt = exp2f(mr - M);
+            L += tab[r * kPartial + 1] * wgt;
+            O += tab[r * kPartial + 4 + e] * wgt;
           }
+          res = O / L;
         }
-        float M = -INFINITY;
-#pragma unroll
-        for (int r = 0; r < kMaxCluster; ++r) M = fmaxf(M, mv[r]);
-        float L = 0.0f, O = 0.0f;
-#pragma unroll
-        for (int r = 0; r < kMaxCluster; ++r) {
-          if (mv[r] == -INFINITY) continue;  // a block that kept no token of this head
-          const float wgt = exp2f(mv[r] - M);
-          L += lv[r] * wgt;
-          O += ov[r] * wgt;
-        }
-        res = O / L;
+        p.out[hq * kDim + e] = res;
       }
-      p.out[hq * kDim + e] = res;
     }
-    for (int i = tid; i < G * p.budget; i += kWorkers) {
-      const int g = i / p.budget, r = i - g * p.budget;
-      if (r >= keff) p.idx[((int64_t)b * p.Hq + kvh * G + g) * p.budget + r] = -1;
-    }
+    if (rank == 0)
+      for (int i = tid; i < G * p.budget; i += kWorkers) {
+        const int g = i / p.budget, r = i - g * p.budget;
+        if (r >= keff) p.idx[((int64_t)b * p.Hq + kvh * G + g) * p.budget + r] = -1;
+      }
   }
-  __syncthreads();
-  cluster.sync();  // peers may still be reading this block's shared memory until here
 }
 
 }  // namespace adamas
