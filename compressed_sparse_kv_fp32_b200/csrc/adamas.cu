@@ -136,7 +136,6 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(const uint16_t* __
 constexpr int kMaxDevices = 64;
 constexpr int kMinTokensPerBlock = 2048;  // fewer tokens per block than this only when the context is short
 constexpr int kOccCache = 64;
-constexpr int kMinCandidates = 1024;      // smaller candidate lists are not worth listing
 
 struct OccEntry {
   const void* fn;
@@ -258,7 +257,6 @@ struct Plan {
   int grid = 0;
   int nstages = kMaxStages;
   int dstride = 64;
-  int clist_cap = 0;  // candidate-list entries per query head
   bool smem_d = true;
   size_t smem = 0;
   size_t ctrl = 0, dspill = 0, total = 0;  // workspace offsets / size
@@ -276,8 +274,7 @@ static int check_shape(int B, int Hq, int Hkv, int64_t Nmax, int d, int budget) 
 }
 
 // Shared-memory layout for `cluster` blocks per head: distances in shared memory
-// with as many ring stages as fit, else in the workspace with a full ring; the
-// candidate lists take what is left.
+// with as many ring stages as fit, else in the workspace with a full ring.
 static bool layout_for(int G, int64_t Nmax, int cluster, size_t optin, Plan* P) {
   const int64_t seg_cap = (Nmax + cluster - 1) / cluster;  // tokens of any block
   if (seg_cap >= (int64_t(1) << 23)) return false;          // token offsets are packed in 23 bits
@@ -287,7 +284,7 @@ static bool layout_for(int G, int64_t Nmax, int cluster, size_t optin, Plan* P) 
   for (int pass = 0; pass < 2 && !found; ++pass) {
     const bool in_smem = pass == 0;
     for (int ns = kMaxStages; ns >= kMinStages && !found; --ns) {
-      const size_t s = DecodeSmem::total(G, cluster, ns, P->dstride, in_smem, 0);
+      const size_t s = DecodeSmem::total(G, cluster, ns, P->dstride, in_smem);
       if (s <= optin) {
         P->smem_d = in_smem;
         P->nstages = ns;
@@ -297,16 +294,6 @@ static bool layout_for(int G, int64_t Nmax, int cluster, size_t optin, Plan* P) 
     }
   }
   if (!found) return false;
-  P->clist_cap = 0;
-  if (seg_cap <= kCandMaxTokens) {
-    int64_t cap = (int64_t)(optin - P->smem) / (2 * G);
-    if (cap > P->dstride) cap = P->dstride;
-    cap = cap / 64 * 64;
-    if (cap >= kMinCandidates) {
-      P->clist_cap = (int)cap;
-      P->smem = DecodeSmem::total(G, cluster, P->nstages, P->dstride, P->smem_d, P->clist_cap);
-    }
-  }
   return true;
 }
 
@@ -405,7 +392,6 @@ static int enqueue_decode(const void* q, const uint8_t* codes, const void* K, co
   prm.cluster = P.cluster;
   prm.nstages = P.nstages;
   prm.dstride = P.dstride;
-  prm.clist_cap = P.clist_cap;
   int rc;
   switch (P.G) {
     case 1: rc = launch_decode<1>(prm, P, st); break;

@@ -18,13 +18,8 @@
 //            the kv head, then score every row against them (exact L1, two rows
 //            per thread per stage), keep the G distances of every token (shared
 //            memory, or the workspace when they do not fit) and count them in one
-//            385-bin histogram per query head.  They also list the tokens that
-//            can still be selected: a further warp keeps reading the histograms
-//            of the whole cluster so far and publishes the smallest distance B
-//            with at least k_eff tokens at or below it -- the final threshold of
-//            the head can only be <= B -- and only tokens with D <= B are listed.
-//            When the cluster's histograms fit, every block then writes its own
-//            into a table in each peer.
+//            385-bin histogram per query head.  When the cluster's histograms fit,
+//            every block then writes its own into a table in each peer.
 //   -- cluster barrier --
 //   phase 2  per query head: the C histograms give the threshold T with
 //            count(D < T) < k_eff <= count(D <= T) and, for every distance d, the
@@ -33,12 +28,14 @@
 //            kept; of the ties D == T this block keeps its first k_eff - base(T)
 //            in index order, so ties go to the lowest indices.  A token's output
 //            slot is its rank base + its rank by index among the block's tokens
-//            of equal distance.  From the candidate list (when it did not
-//            overflow): the listed tokens with D <= T are grouped by distance and
-//            ranked inside their group; otherwise two scans of all the block's
-//            distances find them (counts per warp, then an in-order emit, with a
-//            warp match over 32-entry chunks for the D < T tokens).  Either way
-//            the kept tokens end up in slot order, so both give the same bits.
+//            of equal distance.  One pass over the block's distances puts every
+//            token with D <= T (typically a few hundred) into its distance group
+//            (atomic cursors; each thread walks its own run of positions, lanes
+//            rotated so that a warp's loads spread over the banks), and each
+//            token is then ranked inside its group.  When groups are large (heavy
+//            ties) two scans take over: per-warp counts, then an in-order emit
+//            with a warp match over 32-entry chunks for the D < T tokens.  Either
+//            way the kept tokens end up in slot order, so both give the same bits.
 //            The kept K/V rows are prefetched into L2, gathered into registers
 //            (each half-warp keeps four K and four V rows in flight) and folded
 //            into an online-softmax state per half-warp; the states become one
@@ -65,11 +62,8 @@ namespace cg = cooperative_groups;
 
 constexpr int kWorkers = 512;                         // scoring / select / gather threads
 constexpr int kWorkerWarps = kWorkers / 32;
-constexpr int kCopyWarp = kWorkerWarps;               // issues the bulk copies of the code stream
-constexpr int kBoundWarp = kWorkerWarps + 1;          // keeps the candidate bounds of phase 1 tight
-constexpr int kThreads = kWorkers + 64;
-constexpr int kBoundRounds = 4096;                    // most bound updates of one step
-constexpr int kStageRows = 1024;                      // code rows per ring stage
+constexpr int kThreads = kWorkers + 32;               // + the warp that issues the bulk copies
+constexpr int kStageRows = 2 * kWorkers;              // code rows per ring stage (two per worker)
 constexpr uint32_t kStageBytes = kStageRows * kCodeBytes;  // 32 KiB
 constexpr int kRowsPerThread = kStageRows / kWorkers;
 constexpr int kMaxStages = 4;
@@ -77,17 +71,15 @@ constexpr int kMinStages = 2;
 constexpr int kMaxCluster = 16;
 constexpr int kHistStride = 388;                      // >= kBins, multiple of 4
 constexpr int kPartial = 132;                         // m, l, pad, pad, o[128]
-constexpr int kListCap = 4096;                        // D < T tokens listed per round / grouped candidates
+constexpr int kListCap = 4096;                        // D < T tokens listed per round / grouped tokens D <= T
 constexpr int kKeptCap = 4096;                        // kept tokens per gather window
-constexpr int kGroupMax = 512;                        // largest equal-distance group ranked from the candidate list
-constexpr int kCandMaxTokens = 65535;                 // candidate-list positions are 16-bit
+constexpr int kGroupMax = 512;                        // largest equal-distance group ranked pairwise
 constexpr int kGatherRows = 4;                        // K/V rows in flight per half-warp
 constexpr int kScanBatch = 4;                         // 32-group iterations of a distance scan loaded together
 constexpr int kGatherBatch = 2 * kWorkerWarps * kGatherRows;  // rows per gather batch of the block
 constexpr int kPushHistMax = 8;                       // C * G up to which histograms are pushed to peers
 constexpr uint32_t kPosMask = (1u << 23) - 1u;        // token offset within a block (list entries: d << 23 | t)
 constexpr uint32_t kWaitLimit = 1u << 20;             // mbarrier polls (about a second)
-constexpr int kNoBound = 0x7FFF;                      // candidate bound before the block has k_eff tokens
 
 struct DecodeParams {
   const uint16_t* q;
@@ -105,7 +97,6 @@ struct DecodeParams {
   int cluster;          // blocks per (b, kv head)
   int nstages;          // ring stages, kMinStages..kMaxStages
   int dstride;          // distances per query head and block (>= any block's tokens, multiple of 64)
-  int clist_cap;        // candidate-list entries per query head (0: no candidate list)
 };
 
 // Shared-memory carve-up (bytes), shared with the host.
@@ -117,7 +108,6 @@ struct DecodeParams {
 //          (later the half-warp softmax states), carried counts / group cursors
 //          [kHistStride], D < T tokens or grouped candidates [kListCap], kept tokens [kKeptCap]
 //   dist:  [G][dstride] u16 when kept in shared memory
-//   clist: [G][clist_cap] u16 candidate positions
 struct DecodeSmem {
   static __host__ __device__ inline size_t align128(size_t x) { return (x + 127) / 128 * 128; }
   static __host__ __device__ inline bool push_hist(int G, int C) { return G * C <= kPushHistMax; }
@@ -141,9 +131,8 @@ struct DecodeSmem {
   static __host__ __device__ inline size_t dist(int G, int dstride, bool in_smem) {
     return in_smem ? align128((size_t)G * dstride * 2) : 0;
   }
-  static __host__ __device__ inline size_t clist(int G, int cap) { return align128((size_t)G * cap * 2); }
-  static __host__ __device__ inline size_t total(int G, int C, int nstages, int dstride, bool in_smem, int cap) {
-    return head(G, C) + ring(nstages) + dist(G, dstride, in_smem) + clist(G, cap);
+  static __host__ __device__ inline size_t total(int G, int C, int nstages, int dstride, bool in_smem) {
+    return head(G, C) + ring(nstages) + dist(G, dstride, in_smem);
   }
 };
 static_assert(DecodeSmem::cnt() >= DecodeSmem::state(), "softmax states overlay the chunk counts");
@@ -151,7 +140,7 @@ static_assert(DecodeSmem::cnt() + DecodeSmem::carry() + (kListCap + kKeptCap) * 
               "phase-2 arrays fit in the smallest ring");
 
 // ------------------------------------------------------------------ block helpers
-// Barrier of the sixteen worker warps (the copy warp does not take part).
+// Barrier of the worker warps (the copy warp does not take part).
 __device__ __forceinline__ void worker_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kWorkers) : "memory"); }
 
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
@@ -184,42 +173,6 @@ __device__ __forceinline__ int warp_inclusive_scan(int x, int lane) {
     if (lane >= o) x += y;
   }
   return x;
-}
-
-// Smallest distance B with at least k tokens of the cluster's head at or below
-// it, from histograms that their blocks may still be adding to (any snapshot of
-// the counts gives a valid B, as every count read is of real tokens); -1 while
-// fewer than k tokens are counted.  Whole warp.  `hist` is this block's
-// histogram; with peers, the same histogram of every block of the cluster is
-// read (relaxed cluster-scope loads, all of a block's in flight together).
-__device__ __forceinline__ int kth_bound(const uint32_t* hist, int C, bool peers, int rank, int k, int lane) {
-  constexpr int kPer = (kBins + 31) / 32;
-  const uint32_t a0 = smem_addr(hist) + (uint32_t)(lane * kPer) * 4u;
-  int cnt[kPer];
-#pragma unroll
-  for (int i = 0; i < kPer; ++i) cnt[i] = 0;
-  for (int r = 0; r < (peers ? C : 1); ++r) {
-    const uint32_t a = mapa_shared(a0, peers ? r : rank);
-    uint32_t v[kPer];
-#pragma unroll
-    for (int i = 0; i < kPer; ++i) v[i] = lane * kPer + i < kBins ? ld_relaxed_cluster(a + 4u * i) : 0u;
-#pragma unroll
-    for (int i = 0; i < kPer; ++i) cnt[i] += (int)v[i];
-  }
-  int s = 0;
-#pragma unroll
-  for (int i = 0; i < kPer; ++i) s += cnt[i];
-  const int incl = warp_inclusive_scan(s, lane);
-  const uint32_t crossed = __ballot_sync(0xffffffffu, incl >= k);
-  if (crossed == 0u) return -1;
-  const int L = __ffs((int)crossed) - 1;
-  int res = 0, run = incl - s;
-#pragma unroll
-  for (int i = 0; i < kPer; ++i) {
-    run += cnt[i];
-    if (run >= k && res == 0 && lane == L) res = lane * kPer + i + 1;
-  }
-  return __shfl_sync(0xffffffffu, res, L) - 1;
 }
 
 // Eight consecutive distances 8*grp .. 8*grp+7 as four words of u16 pairs (element
@@ -346,9 +299,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const DecodePa
   __shared__ __align__(8) uint64_t sm_full[kMaxStages];
   __shared__ __align__(8) uint64_t sm_empty[kMaxStages];
   __shared__ int sm_T[kMaxGroup];
-  __shared__ int sm_bound[kMaxGroup];   // candidate bound per query head (phase 1)
-  __shared__ int sm_scored;             // a worker warp has scored all its rows
-  __shared__ int sm_ncand[kMaxGroup][kWorkerWarps];  // candidates listed per query head and warp (may exceed the capacity)
   __shared__ int sm_wlt[kWorkerWarps];  // per warp: candidates with D < T
   __shared__ int sm_weq[kWorkerWarps];  // per warp: candidates with D == T
   __shared__ int sm_wmax[kWorkerWarps];
@@ -363,9 +313,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const DecodePa
   const bool worker = warp < kWorkerWarps;
   const uint32_t lt = (1u << lane) - 1u;
   const bool push_hist = DecodeSmem::push_hist(G, C);
-  const int ccap = p.clist_cap;              // per query head: kWorkerWarps lists of wcap entries
-  const int wcap = ccap / kWorkerWarps;
-  const bool use_cand = ccap > 0;
 
   unsigned char* cur = smem;
   uint32_t* sm_q = reinterpret_cast<uint32_t*>(cur);      cur += DecodeSmem::qcodes(G);    // [G][8]
@@ -383,7 +330,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const DecodePa
   } else {
     dist = p.dglobal + (size_t)blockIdx.x * G * p.dstride;
   }
-  uint16_t* sm_cand = reinterpret_cast<uint16_t*>(cur);  // [G][kWorkerWarps][wcap]
   // phase-2 arrays over the ring
   uint32_t* sm_cnt = reinterpret_cast<uint32_t*>(ring);                          // [kWorkerWarps][kHistStride]
   float* sm_state = reinterpret_cast<float*>(ring);                              // [2*kWorkerWarps][kPartial]
@@ -412,37 +358,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const DecodePa
     fence_mbar_init();
   }
   for (int i = tid; i < G * kHistStride; i += kThreads) sm_hist[i] = 0u;
-  if (tid < kMaxGroup) {
-    sm_T[tid] = kBins - 1;  // always overwritten when the histograms are consistent
-    sm_bound[tid] = kNoBound;
-  }
-  if (tid == 0) sm_scored = 0;
+  if (tid < kMaxGroup) sm_T[tid] = kBins - 1;  // always overwritten when the histograms are consistent
   __syncthreads();
-  // Peers read this block's histograms during phase 1 (candidate bounds): every
-  // thread arrives on a cluster barrier once the histograms are cleared and waits
-  // on it before it (or a peer, in turn) can look at another block -- after the
-  // first stage, long after every block has arrived.
+  // Every block of the cluster has started (and may be written to through
+  // distributed shared memory) once every thread has arrived here; each thread
+  // waits on it before its first such access.
   cluster_arrive();
-  bool waited = false;
 
   // ================================================================ phase 1
-  if (warp == kBoundWarp) {
-    // Recompute the candidate bounds from the whole cluster's histograms until the
-    // stream is scored; the workers only read them.
-    cluster_wait();
-    waited = true;
-    if (use_cand && nst > 0)
-      for (int it = 0; it < kBoundRounds; ++it) {
-        if (*(volatile int*)&sm_scored) break;
-#pragma unroll 1
-        for (int g = 0; g < G; ++g) {
-          const int bnd = kth_bound(sm_hist + g * kHistStride, C, true, rank, keff, lane);
-          if (bnd >= 0 && lane == 0) atomicMin(&sm_bound[g], bnd);
-        }
-        __syncwarp();
-        __nanosleep(500);
-      }
-  } else if (!worker) {
+  if (!worker) {
     if (lane == 0) {
       const unsigned char* src = p.codes + (kv_base + t0) * kCodeBytes;
       for (int i = 0; i < nst; ++i) {
@@ -455,6 +379,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const DecodePa
       }
     }
     __syncwarp();
+    cluster_wait();
   } else {
     if (warp < G && keff > 0) {
       const uint32_t w = encode128_warp(p.q + ((int64_t)b * p.Hq + kvh * G + warp) * kDim, lane);
@@ -476,28 +401,29 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const DecodePa
           rm[g][w] = sm_qc[g * 2 * kCodeWords + kCodeWords + w];
         }
     }
-    int ncand[G];  // this warp's listed candidates per query head (uniform in the warp)
-#pragma unroll
-    for (int g = 0; g < G; ++g) ncand[g] = 0;
     for (int i = 0; i < nst; ++i) {
       const int buf = i % NS;
       if (!mbar_wait(&sm_full[buf], (uint32_t)(i / NS) & 1u, kWaitLimit)) atomicOr(p.err, kErrTimeout);
       const int rows = min(kStageRows, seg_len - i * kStageRows);
       const unsigned char* st = ring + (size_t)buf * kStageBytes;
-      int bound[G];
+      uint4 kx[kRowsPerThread][2];
 #pragma unroll
-      for (int g = 0; g < G; ++g) bound[g] = use_cand ? *(volatile int*)&sm_bound[g] : -1;
-      int dg[kRowsPerThread][G];  // kNoBound + 1 for rows past the stage's end
+      for (int j = 0; j < kRowsPerThread; ++j) {
+        const int r = j * kWorkers + tid;
+        kx[j][0] = make_uint4(0u, 0u, 0u, 0u);
+        kx[j][1] = kx[j][0];
+        if (r < rows) {
+          const uint32_t ra = smem_addr(st + (size_t)r * kCodeBytes);
+          kx[j][0] = lds128(ra);
+          kx[j][1] = lds128(ra + 16);
+        }
+      }
 #pragma unroll
       for (int j = 0; j < kRowsPerThread; ++j) {
         const int r = j * kWorkers + tid;
         const int t = i * kStageRows + r;
-#pragma unroll
-        for (int g = 0; g < G; ++g) dg[j][g] = kNoBound + 1;
         if (r < rows) {
-          const uint32_t ra = smem_addr(st + (size_t)r * kCodeBytes);
-          const uint4 x0 = lds128(ra);
-          const uint4 x1 = lds128(ra + 16);
+          const uint4 x0 = kx[j][0], x1 = kx[j][1];
           const uint32_t k[kCodeWords] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
           uint32_t k1[kCodeWords];
           key_shift(k, k1);
@@ -516,33 +442,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const DecodePa
               mg[4] = m1.x; mg[5] = m1.y; mg[6] = m1.z; mg[7] = m1.w;
               d = l1_distance(k, k1, qg, mg);
             }
-            dg[j][g] = d;
             if constexpr (SMEM_D) sts16(smem_addr(dist + (size_t)g * p.dstride + t), (uint16_t)d);
             else dist[(size_t)g * p.dstride + t] = (uint16_t)d;
             atomicAdd(&sm_hist[g * kHistStride + d], 1u);
           }
         }
       }
-      if (use_cand) {
-#pragma unroll
-        for (int j = 0; j < kRowsPerThread; ++j)
-#pragma unroll
-          for (int g = 0; g < G; ++g) {  // list the row if it can still be selected
-            const bool pred = dg[j][g] <= bound[g];
-            const uint32_t m = __ballot_sync(0xffffffffu, pred);
-            const int at = ncand[g] + __popc(m & lt);
-            if (pred && at < wcap)
-              sm_cand[(size_t)g * ccap + warp * wcap + at] = (uint16_t)(i * kStageRows + j * kWorkers + tid);
-            ncand[g] += __popc(m);
-          }
-      }
+      // Every lane has used its rows: only now does the stage go back to the copy warp
+      // (one arrive per warp after __syncwarp does not order other lanes' loads that
+      // are still in flight against the refill).
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm_empty[buf]);
     }
-    if (lane == 0) *(volatile int*)&sm_scored = 1;
-    if (lane == 0)
-#pragma unroll
-      for (int g = 0; g < G; ++g) sm_ncand[g][warp] = ncand[g];
+
+    cluster_wait();
     if (push_hist && keff > 0) {  // own histograms into every block's table (row `rank`)
       worker_sync();
       for (int r = 0; r < C; ++r) {
@@ -551,7 +464,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const DecodePa
       }
     }
   }
-  if (!waited) cluster_wait();
   __syncthreads();
   cluster.sync();  // every block's histograms are complete and visible to the cluster
 
@@ -594,7 +506,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const DecodePa
     }
     worker_sync();
 
-    const int hw = tid >> 4, hl = tid & 15;  // 32 half-warps
+    const int hw = tid >> 4, hl = tid & 15;  // two half-warps per worker warp
     const float kScoreScale = 0.08838834764831845f * 1.4426950408889634f;  // log2(e)/sqrt(128)
     // warp slices over 8-position groups of the block's distances (full scans)
     const int ngrp = (seg_len + 7) >> 3;
@@ -624,14 +536,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const DecodePa
       }
       for (int i = tid; i < kHistStride; i += kWorkers) sm_carry[i] = 0u;
       worker_sync();
-      int gmax = 0, cmax = 0;
+      int gmax = 0;
 #pragma unroll
-      for (int w = 0; w < kWorkerWarps; ++w) {
-        gmax = max(gmax, sm_wmax[w]);
-        cmax = max(cmax, sm_ncand[g][w]);
-      }
-      bool from_list = use_cand && cmax <= wcap && n_lt + n_eq <= kListCap && n_kept <= kKeptCap &&
-                       gmax <= kGroupMax;
+      for (int w = 0; w < kWorkerWarps; ++w) gmax = max(gmax, sm_wmax[w]);
+      // grouped path: every token with D <= T grouped by distance and ranked inside
+      // its group; else the two scans
+      bool grouped = n_lt + n_eq <= kListCap && n_kept <= kKeptCap && gmax <= kGroupMax;
 
       float qf[8];
       float m_run = -INFINITY, l_run = 0.0f, o[8];
@@ -651,17 +561,29 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const DecodePa
         }
       };
 
-      if (from_list) {
-        // ---- candidates with D <= T grouped by distance (group d at [lpre[d], lpre[d] + hist[d]))
-        const uint16_t* cand = sm_cand + (size_t)g * ccap + warp * wcap;  // this warp's phase-1 list
-        const int nw = sm_ncand[g][warp];
-        for (int x = lane; x < nw; x += 32) {
-          uint16_t tpos;
-          asm volatile("ld.shared.u16 %0, [%1];" : "=h"(tpos) : "r"(smem_addr(cand + x)) : "memory");
-          const uint32_t d = load_dist1<SMEM_D>(drow, tpos);
-          if (d <= T) {
+      if (grouped) {
+        // ---- every token with D <= T to its group (group d at [lpre[d], lpre[d] + hist[d])):
+        // each thread takes a run of 8-position groups, lanes start at different
+        // points of their runs so that a warp's loads spread over the banks
+        const uint32_t tx2 = T | T << 16, t1x2 = (T + 1) | (T + 1) << 16;
+        const int chunk = (ngrp + kWorkers - 1) / kWorkers;
+        const int rot = lane % chunk;
+        for (int k = 0; k < chunk; ++k) {
+          int kk = k + rot;
+          if (kk >= chunk) kk -= chunk;
+          const int grp = tid * chunk + kk;
+          if (grp >= ngrp) continue;
+          const uint4 v = load_dist8<SMEM_D>(drow, grp);
+          if (!any_le(v, t1x2)) continue;
+          uint32_t mlt, meq;
+          cand_bits(v, tx2, t1x2, mlt, meq);
+          for (uint32_t m = mlt | meq; m != 0u; m &= m - 1u) {
+            const int e = __ffs((int)m) - 1;
+            const uint32_t wv = e < 4 ? (e < 2 ? v.x : v.y) : (e < 6 ? v.z : v.w);
+            const uint32_t d = (wv >> (16 * (e & 1))) & 0xFFFFu;
             const uint32_t c = atomicAdd(&sm_carry[d], 1u);
-            if (c >= hist_g[d]) continue;  // never with a complete list (checked below)
+            if (c >= hist_g[d]) continue;  // never with consistent histograms (checked below)
+            const uint32_t tpos = (uint32_t)(grp * 8 + e);
             sm_list[lpre_g[d] + c] = (int32_t)(d << 23 | tpos);
             const int64_t row = kv_base + t0 + tpos;  // the row is very likely kept: on its way into L2
             prefetch_l2(p.K + row * kDim);
@@ -671,15 +593,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const DecodePa
           }
         }
         worker_sync();
-        // every group must be complete (each token with D <= T listed once), else the scans decide
+        // every group must be complete (each token with D <= T placed once), else the scans decide
         if (tid == 0) sm_wmax[0] = 0;
         worker_sync();
         if (tid <= (int)T && sm_carry[tid] != hist_g[tid]) sm_wmax[0] = 1;
         worker_sync();
-        from_list = sm_wmax[0] == 0;
+        grouped = sm_wmax[0] == 0;
         worker_sync();
       }
-      if (from_list) {
+      if (grouped) {
         // ---- rank inside the group by index: slot, and the kept position lpre[d] + rank
         const int nf = n_lt + n_eq;
         for (int i = tid; i < nf; i += kWorkers) {
@@ -702,7 +624,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const DecodePa
         gather(n_kept, false);
         worker_sync();
       }
-      if (!from_list) {
+      if (!grouped) {
         // ---- count pass: candidates per warp
         const uint32_t tx2 = T | T << 16, t1x2 = (T + 1) | (T + 1) << 16;
         int c_lt = 0, c_eq = 0;
