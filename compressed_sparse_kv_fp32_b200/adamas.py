@@ -30,7 +30,7 @@ _lib = None
 SYMBOLS = (
     "adamas_status_string", "adamas_version", "adamas_last_error_string", "adamas_workspace_bytes", "adamas_workspace_init",
     "adamas_encode_keys", "adamas_decode_step", "adamas_score", "adamas_get_device_error",
-    "adamas_decode_step_static",
+    "adamas_decode_step_static", "adamas_decode_step_append",
 )
 
 
@@ -71,6 +71,8 @@ def load(path: str = LIBRARY) -> ctypes.CDLL:
         l.adamas_get_device_error.restype = I
         l.adamas_decode_step_static.argtypes = [P, P, P, P, P, I, I, I, I64, I, I, P, P, P]
         l.adamas_decode_step_static.restype = I
+        l.adamas_decode_step_append.argtypes = [P, P, P, P, P, P, I, I, I, I64, I, I, P, P, P, SZ, P]
+        l.adamas_decode_step_append.restype = I
         _lib = l
         return l
 
@@ -154,11 +156,7 @@ def encode_keys(K: torch.Tensor, codes: torch.Tensor, pos_begin: Optional[torch.
     return codes
 
 
-def decode_step(q: torch.Tensor, codes: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
-                seq_lens: torch.Tensor, budget: int, workspace: Workspace,
-                out: Optional[torch.Tensor] = None, idx: Optional[torch.Tensor] = None,
-                stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor]:
-    """One decode step: returns (out [B,Hq,128] fp32, idx [B,Hq,budget] int32)."""
+def _decode_args(q, codes, K, V, seq_lens, budget, out, idx):
     _need(q, "q", torch.bfloat16)
     if q.dim() != 3:
         raise ValueError("q must be [B, Hq, 128]")
@@ -177,11 +175,36 @@ def decode_step(q: torch.Tensor, codes: torch.Tensor, K: torch.Tensor, V: torch.
         idx = torch.empty((B, Hq, budget), dtype=torch.int32, device=q.device)
     _need(out, "out", torch.float32, (B, Hq, d))
     _need(idx, "idx", torch.int32, (B, Hq, budget))
+    return B, Hq, Hkv, Nmax, d, out, idx
+
+
+def decode_step(q: torch.Tensor, codes: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
+                seq_lens: torch.Tensor, budget: int, workspace: Workspace,
+                out: Optional[torch.Tensor] = None, idx: Optional[torch.Tensor] = None,
+                stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """One decode step: returns (out [B,Hq,128] fp32, idx [B,Hq,budget] int32)."""
+    B, Hq, Hkv, Nmax, d, out, idx = _decode_args(q, codes, K, V, seq_lens, budget, out, idx)
     rc = load().adamas_decode_step(q.data_ptr(), codes.data_ptr(), K.data_ptr(), V.data_ptr(),
                                    seq_lens.data_ptr(), B, Hq, Hkv, Nmax, d, budget, out.data_ptr(),
                                    idx.data_ptr() if budget > 0 else None,
                                    workspace.buffer.data_ptr(), workspace.nbytes, _stream(stream))
     _check(rc, "adamas_decode_step")
+    return out, idx
+
+
+def decode_step_append(q: torch.Tensor, codes: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
+                       seq_lens: torch.Tensor, append_pos: torch.Tensor, budget: int, workspace: Workspace,
+                       out: Optional[torch.Tensor] = None, idx: Optional[torch.Tensor] = None,
+                       stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """encode_keys of the key at append_pos[b] (int32 [B]; out of [0, Nmax): none)
+    followed by decode_step, in one launch; codes is updated in place."""
+    B, Hq, Hkv, Nmax, d, out, idx = _decode_args(q, codes, K, V, seq_lens, budget, out, idx)
+    _need(append_pos, "append_pos", torch.int32, (B,))
+    rc = load().adamas_decode_step_append(q.data_ptr(), codes.data_ptr(), K.data_ptr(), V.data_ptr(),
+                                          seq_lens.data_ptr(), append_pos.data_ptr(), B, Hq, Hkv, Nmax, d,
+                                          budget, out.data_ptr(), idx.data_ptr() if budget > 0 else None,
+                                          workspace.buffer.data_ptr(), workspace.nbytes, _stream(stream))
+    _check(rc, "adamas_decode_step_append")
     return out, idx
 
 

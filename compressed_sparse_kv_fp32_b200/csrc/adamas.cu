@@ -370,10 +370,12 @@ static int check_decode_args(const void* q, const uint8_t* codes, const void* K,
   return ADAMAS_OK;
 }
 
-// Enqueue the decode kernel with its scratch at `ws` (laid out by `P`).
+// Enqueue the decode kernel with its scratch at `ws` (laid out by `P`); with
+// append_pos, the keys at those positions are encoded into codes first.
 static int enqueue_decode(const void* q, const uint8_t* codes, const void* K, const void* V,
                           const int32_t* seq_lens, int B, int Hq, int Hkv, int64_t Nmax, int budget, float* out,
-                          int32_t* idx, unsigned char* ws, const Plan& P, cudaStream_t st) {
+                          int32_t* idx, unsigned char* ws, const Plan& P, cudaStream_t st,
+                          const int32_t* append_pos = nullptr) {
   DecodeParams prm;
   prm.q = static_cast<const uint16_t*>(q);
   prm.codes = codes;
@@ -384,6 +386,8 @@ static int enqueue_decode(const void* q, const uint8_t* codes, const void* K, co
   prm.idx = idx;
   prm.err = reinterpret_cast<uint32_t*>(ws + P.ctrl) + 2;
   prm.dglobal = P.smem_d ? nullptr : reinterpret_cast<uint16_t*>(ws + P.dspill);
+  prm.codes_w = append_pos ? const_cast<uint8_t*>(codes) : nullptr;
+  prm.append_pos = append_pos;
   prm.B = B;
   prm.Hq = Hq;
   prm.Hkv = Hkv;
@@ -493,6 +497,24 @@ int adamas_decode_step(const void* q, const uint8_t* codes, const void* K, const
   if (!workspace || workspace_bytes < P.total || !aligned(workspace, 16)) return ADAMAS_ERR_WORKSPACE;
   return enqueue_decode(q, codes, K, V, seq_lens, B, Hq, Hkv, Nmax, budget, out, idx,
                         static_cast<unsigned char*>(workspace), P, (cudaStream_t)stream);
+}
+
+int adamas_decode_step_append(const void* q, uint8_t* codes, const void* K, const void* V, const int32_t* seq_lens,
+                              const int32_t* append_pos, int B, int Hq, int Hkv, int64_t Nmax, int d, int budget,
+                              float* out, int32_t* idx, void* workspace, size_t workspace_bytes,
+                              adamas_stream_t stream) {
+  int rc = check_decode_args(q, codes, K, V, seq_lens, B, Hq, Hkv, Nmax, d, budget, out, idx);
+  if (rc != ADAMAS_OK || B == 0) return rc;
+  if (!append_pos || !aligned(append_pos, 4)) return ADAMAS_ERR_INVALID_ARG;
+  if (Nmax == 0) return adamas_decode_step(q, codes, K, V, seq_lens, B, Hq, Hkv, Nmax, d, budget, out, idx, workspace,
+                                           workspace_bytes, stream);
+  DeviceInfo* dev = nullptr;
+  if ((rc = device_info(&dev)) != ADAMAS_OK) return rc;
+  Plan P;
+  if ((rc = make_plan(B, Hq, Hkv, Nmax, *dev, &P)) != ADAMAS_OK) return rc;
+  if (!workspace || workspace_bytes < P.total || !aligned(workspace, 16)) return ADAMAS_ERR_WORKSPACE;
+  return enqueue_decode(q, codes, K, V, seq_lens, B, Hq, Hkv, Nmax, budget, out, idx,
+                        static_cast<unsigned char*>(workspace), P, (cudaStream_t)stream, append_pos);
 }
 
 int adamas_score(const void* q, const uint8_t* codes, const int32_t* seq_lens, int B, int Hq, int Hkv, int64_t Nmax,

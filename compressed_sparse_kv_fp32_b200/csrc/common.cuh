@@ -78,16 +78,6 @@ __device__ __forceinline__ uint32_t ld_relaxed_cluster(uint32_t a) {
 __device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release;" ::: "memory"); }
 __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire;" ::: "memory"); }
 
-// Release add / acquire load on a shared-memory counter (CTA scope).
-__device__ __forceinline__ void red_release_cta_add(uint32_t a, uint32_t v) {
-  asm volatile("red.release.cta.shared::cta.add.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
-}
-__device__ __forceinline__ uint32_t ld_acquire_cta(uint32_t a) {
-  uint32_t v;
-  asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
-  return v;
-}
-
 __device__ __forceinline__ void sts16(uint32_t a, uint16_t v) {
   asm volatile("st.shared.u16 [%0], %1;" ::"r"(a), "h"(v) : "memory");
 }
@@ -99,12 +89,6 @@ __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
 // Make initialised barriers visible to the async (bulk copy) proxy.
 __device__ __forceinline__ void fence_mbar_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-
-// Order this thread's earlier generic-proxy shared-memory accesses before later
-// async-proxy (bulk copy) accesses.
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {

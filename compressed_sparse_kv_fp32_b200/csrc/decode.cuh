@@ -91,6 +91,8 @@ struct DecodeParams {
   int32_t* idx;
   uint32_t* err;        // device error word
   uint16_t* dglobal;    // [grid][G][dstride] when distances do not fit in shared memory
+  uint8_t* codes_w;     // writable codes when appending (the same array as codes), else null
+  const int32_t* append_pos;  // [B] position whose key is encoded before scoring (null: none)
   int B, Hq, Hkv;
   int64_t Nmax;
   int budget;
@@ -302,6 +304,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const DecodePa
   __shared__ int sm_wlt[kWorkerWarps];  // per warp: candidates with D < T
   __shared__ int sm_weq[kWorkerWarps];  // per warp: candidates with D == T
   __shared__ int sm_wmax[kWorkerWarps];
+  __shared__ uint32_t sm_acode[kCodeWords];  // the appended key's code
   __shared__ long long sm_tmp[kWorkerWarps];
 
   cg::cluster_group cluster = cg::this_cluster();
@@ -337,8 +340,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const DecodePa
   int32_t* sm_list = reinterpret_cast<int32_t*>(ring + DecodeSmem::cnt() + DecodeSmem::carry());  // [kListCap]
   int32_t* sm_kept = sm_list + kListCap;                                         // [kKeptCap]
 
-  // ---- the head's length and this block's tokens
+  // ---- the head's length and this block's tokens (both loads in flight together)
+  const int32_t* ap_src = p.append_pos ? p.append_pos + b : p.seq_lens + b;
   int64_t len_b = p.seq_lens[b];
+  const int32_t ap_raw = *ap_src;
+  const int64_t ap = p.append_pos ? ap_raw : -1;
   if (len_b < 0 || len_b > p.Nmax) {
     if (rank == 0 && tid == 0) atomicOr(p.err, kErrSeqLen);
     len_b = len_b < 0 ? 0 : p.Nmax;
@@ -349,6 +355,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const DecodePa
   const int NS = p.nstages;
   const int nst = keff > 0 ? (seg_len + kStageRows - 1) / kStageRows : 0;  // nothing to score without a budget
   const int64_t kv_base = (int64_t)hk * p.Nmax;
+  // appended key of this (b, kv head): encoded by a spare worker warp of the block
+  // that owns its position (the last block when it lies past the sequence) while
+  // the query is encoded.  The code goes to the cache and to shared memory; the
+  // stage copy may carry the cache row's old or new bytes, and the workers score
+  // the shared-memory copy in its place.
+  int64_t apos = -1;
+  int arow = -1;  // its row in this block's segment (-1: not scored here)
+  if (ap >= 0 && ap < p.Nmax && ((ap >= t0 && ap < t0 + seg_len) || (rank == C - 1 && ap >= len_b))) {
+    apos = ap;
+    if (ap >= t0 && ap < t0 + seg_len) arow = (int)(ap - t0);
+  }
+  const int astage = arow >= 0 ? arow / kStageRows : -1;
 
   if (tid == 0) {
     for (int i = 0; i < NS; ++i) {
@@ -367,17 +385,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const DecodePa
 
   // ================================================================ phase 1
   if (!worker) {
-    if (lane == 0) {
-      const unsigned char* src = p.codes + (kv_base + t0) * kCodeBytes;
-      for (int i = 0; i < nst; ++i) {
-        const int buf = i % NS;
-        if (i >= NS && !mbar_wait(&sm_empty[buf], (uint32_t)((i / NS) - 1) & 1u, kWaitLimit))
-          atomicOr(p.err, kErrTimeout);
-        const uint32_t bytes = (uint32_t)min(kStageRows, seg_len - i * kStageRows) * kCodeBytes;
-        mbar_arrive_expect_tx(&sm_full[buf], bytes);
-        bulk_copy_g2s(ring + (size_t)buf * kStageBytes, src + (size_t)i * kStageBytes, bytes, &sm_full[buf]);
-      }
-    }
+    const unsigned char* src = p.codes + (kv_base + t0) * kCodeBytes;
+    auto issue = [&](int i) {
+      const int buf = i % NS;
+      if (i >= NS && !mbar_wait(&sm_empty[buf], (uint32_t)((i / NS) - 1) & 1u, kWaitLimit))
+        atomicOr(p.err, kErrTimeout);
+      const uint32_t bytes = (uint32_t)min(kStageRows, seg_len - i * kStageRows) * kCodeBytes;
+      mbar_arrive_expect_tx(&sm_full[buf], bytes);
+      bulk_copy_g2s(ring + (size_t)buf * kStageBytes, src + (size_t)i * kStageBytes, bytes, &sm_full[buf]);
+    };
+    if (lane == 0)
+      for (int i = 0; i < nst; ++i) issue(i);
     __syncwarp();
     cluster_wait();
   } else {
@@ -387,6 +405,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const DecodePa
         sm_q[warp * kCodeWords + lane] = w;
         sm_qc[warp * 2 * kCodeWords + lane] = w;
         sm_qc[warp * 2 * kCodeWords + kCodeWords + lane] = query_mask(w);
+      }
+    }
+    if (warp == kWorkerWarps - 1 && apos >= 0) {  // the same encoder as adamas_encode_keys
+      const uint32_t w = encode128_warp(p.K + (kv_base + apos) * kDim, lane);
+      if (lane < kCodeWords) {
+        sm_acode[lane] = w;
+        reinterpret_cast<uint32_t*>(p.codes_w + (kv_base + apos) * kCodeBytes)[lane] = w;
       }
     }
     worker_sync();
@@ -417,6 +442,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const DecodePa
           kx[j][0] = lds128(ra);
           kx[j][1] = lds128(ra + 16);
         }
+      }
+      if (i == astage) {  // the appended row: its fresh code
+#pragma unroll
+        for (int j = 0; j < kRowsPerThread; ++j)
+          if (i * kStageRows + j * kWorkers + tid == arow) {
+            kx[j][0] = make_uint4(sm_acode[0], sm_acode[1], sm_acode[2], sm_acode[3]);
+            kx[j][1] = make_uint4(sm_acode[4], sm_acode[5], sm_acode[6], sm_acode[7]);
+          }
       }
 #pragma unroll
       for (int j = 0; j < kRowsPerThread; ++j) {

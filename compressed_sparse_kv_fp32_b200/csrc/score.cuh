@@ -37,34 +37,16 @@ __device__ __forceinline__ void key_shift(const uint32_t (&k)[kCodeWords], uint3
   for (int w = 0; w < kCodeWords; ++w) k1[w] = k[w] << 1;
 }
 
-#ifndef ADAMAS_L1_SWAR_PAIRS
-#define ADAMAS_L1_SWAR_PAIRS 0
-#endif
-// Word pairs of a row whose fields are summed with plain adds instead of popc
-// (the two run on different pipes).
-constexpr int kSwarPairs = ADAMAS_L1_SWAR_PAIRS;
-
-// Fields of two words (each field 0..3) summed into four bytes (each 0..24).
-__device__ __forceinline__ uint32_t fields_to_bytes(uint32_t fa, uint32_t fb) {
-  const uint32_t na = (fa & 0x33333333u) + ((fa >> 2) & 0x33333333u);  // nibbles 0..6
-  const uint32_t nb = (fb & 0x33333333u) + ((fb >> 2) & 0x33333333u);
-  const uint32_t n = na + nb;                                          // nibbles 0..12
-  return (n & 0x0F0F0F0Fu) + ((n >> 4) & 0x0F0F0F0Fu);
-}
-
 // L1 distance of one key code row (k, k1 = k << 1) to one query code row (q, m).
 __device__ __forceinline__ int l1_distance(const uint32_t (&k)[kCodeWords], const uint32_t (&k1)[kCodeWords],
                                            const uint32_t (&q)[kCodeWords], const uint32_t (&m)[kCodeWords]) {
   int d = 0;
-  uint32_t bytes = 0u;  // byte sums of the pairs summed with adds (each byte <= 96)
 #pragma unroll
   for (int w = 0; w < kCodeWords; w += 2) {
     const uint32_t fa = field_absdiff(k[w], k1[w], q[w], m[w]);
     const uint32_t fb = field_absdiff(k[w + 1], k1[w + 1], q[w + 1], m[w + 1]);
-    if (w / 2 < kSwarPairs) bytes += fields_to_bytes(fa, fb);
-    else d += __popc(fa) + __popc(fb) + __popc((fa & 0xAAAAAAAAu) | ((fb >> 1) & 0x55555555u));
+    d += __popc(fa) + __popc(fb) + __popc((fa & 0xAAAAAAAAu) | ((fb >> 1) & 0x55555555u));
   }
-  if (kSwarPairs > 0) d += (int)__dp4a(bytes, 0x01010101u, 0u);
   return d;
 }
 

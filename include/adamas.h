@@ -128,6 +128,25 @@ int adamas_decode_step(const void *q, const uint8_t *codes, const void *K, const
                        size_t workspace_bytes, adamas_stream_t stream);
 
 /*
+ * adamas_encode_keys for one appended token per sequence followed by
+ * adamas_decode_step, in one launch -- the usual decode-loop step (article §3.1:
+ * the code cache grows by one row per generated token; §2.3, §5.2: the step then
+ * scores and selects over the whole cache).  For every (b, kv head) with
+ * 0 <= append_pos[b] < Nmax, the key K[b][kvh][append_pos[b]] (already written by
+ * the caller) is encoded into codes exactly as adamas_encode_keys would, before
+ * the step scores that position; other values of append_pos[b] append nothing.
+ *   codes       device uint8 [B][Hkv][Nmax][32], read and written
+ *   append_pos  device int32 [B]
+ * Every other argument, result and rule is adamas_decode_step's; the results are
+ * bit-identical to adamas_encode_keys(count 1, pos_begin = append_pos) followed
+ * by adamas_decode_step.
+ */
+int adamas_decode_step_append(const void *q, uint8_t *codes, const void *K, const void *V,
+                              const int32_t *seq_lens, const int32_t *append_pos, int B, int Hq,
+                              int Hkv, int64_t Nmax, int d, int budget, float *out, int32_t *idx,
+                              void *workspace, size_t workspace_bytes, adamas_stream_t stream);
+
+/*
  * Debug and test entry point: the distances the decode step ranks by.
  *   dist  device uint16 [B][Hq][Nmax]: D in [0, 384] for t < seq_lens[b],
  *         0xFFFF past the sequence length.
