@@ -177,6 +177,23 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def max_over_ranks(values, device=None):
+    """Element-wise max of per-rank timings over the process group (identity on one rank)."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def job_value(world: int, steps: int, elapsed_ms: float) -> float:
+    """Whole-job throughput: every rank runs `steps` steps of its own replica."""
+    return world * steps / (elapsed_ms / 1e3)
+
+
 # ---------------------------------------------------------------- GPU arm
 def run_gpu(args, rank, world):
     import torch
@@ -275,10 +292,7 @@ def run_gpu(args, rank, world):
         if L["ws"].device_error() != 0:
             raise RuntimeError("device error word set during the bench")
 
-    if world > 1:
-        tt = torch.tensor([elapsed_ms, dec_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        elapsed_ms, dec_ms = float(tt[0]), float(tt[1])
+    elapsed_ms, dec_ms = max_over_ranks([elapsed_ms, dec_ms], dev)
 
     # ---- end to end through the Python API: pinned host inputs in, results out, every step
     e2e_steps = min(args.e2e_steps, K_steps)
@@ -317,15 +331,12 @@ def run_gpu(args, rank, world):
     e1.record()
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) if e2e_steps > 0 else float("nan")
-    if world > 1:
-        tt = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt[0])
+    (e2e_ms,) = max_over_ranks([e2e_ms], dev)
 
     if rank != 0:
         return
     ms_per_step = elapsed_ms / K_steps
-    value = world * K_steps / (elapsed_ms / 1e3)
+    value = job_value(world, K_steps, elapsed_ms)
     step_bytes = accounting.decode_step_bytes([ctx] * B, Hq, Hkv, BUDGET, d)
     enc_bytes = B * Hkv * accounting.encode_bytes_per_vector(d)
     peak, peak_kind = measured_peak()
@@ -344,7 +355,7 @@ def run_gpu(args, rank, world):
                      "unit": "GB/s", "frac": achieved_dec / peak, "traffic": traffic,
                      "algorithmic_bytes_per_launch": launch_bytes, "avg_launch_us": dec_ms * 1e3,
                      "peak_source": f"MEASURED_PEAKS.json hbm_gbs ({peak_kind})"},
-        "e2e": ({"value": world * e2e_steps / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+        "e2e": ({"value": job_value(world, e2e_steps, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                  "d2h_bytes_per_step": d2h} if e2e_steps > 0 else None),
         "gpu_launches": K_steps,
         "clocks": clocks,

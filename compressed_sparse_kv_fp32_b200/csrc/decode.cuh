@@ -351,7 +351,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const DecodePa
   }
   const int keff = (int)min((int64_t)p.budget, len_b);
   const int64_t t0 = (int64_t)rank * len_b / C;
-  const int seg_len = (int)((int64_t)(rank + 1) * len_b / C - t0);  // <= dstride (host sizing)
+  int seg_len = (int)((int64_t)(rank + 1) * len_b / C - t0);  // <= dstride by the host's sizing
+  if (seg_len > p.dstride) {  // never with the host's plan; keeps every distance store in bounds
+    if (tid == 0) atomicOr(p.err, kErrInternal);
+    seg_len = p.dstride;
+  }
   const int NS = p.nstages;
   const int nst = keff > 0 ? (seg_len + kStageRows - 1) / kStageRows : 0;  // nothing to score without a budget
   const int64_t kv_base = (int64_t)hk * p.Nmax;

@@ -63,7 +63,7 @@ enum adamas_status {
 
 /* Bits of the device error word. */
 #define ADAMAS_DEVERR_SEQLEN 0x1u  /* a seq_lens entry was outside [0, Nmax]; it was clamped */
-#define ADAMAS_DEVERR_TIMEOUT 0x2u /* a grid-wide wait gave up; the step's outputs are invalid */
+#define ADAMAS_DEVERR_TIMEOUT 0x2u /* a bounded wait on a stage copy gave up; the step's outputs are invalid */
 #define ADAMAS_DEVERR_INTERNAL 0x4u /* a block's share exceeded its planned size; outputs are invalid */
 
 /* Static description of a status code (never NULL). */
@@ -79,8 +79,9 @@ const char *adamas_last_error_string(void);
 /*
  * Bytes of device workspace adamas_decode_step needs for these sizes on the
  * current CUDA device (0 when the sizes are unsupported).  The workspace holds
- * per-block token histograms, partial softmax states, grid-wait counters and
- * the error word.  It must be zero-filled once before its first use
+ * the device error word and, only when a block's token distances do not fit in
+ * shared memory (very long contexts), a spill area for them; histograms and
+ * partial softmax states stay on chip.  It must be zero-filled once before its first use
  * (adamas_workspace_init); every step leaves it ready for the next one.  One
  * workspace must not be used by two steps that may run concurrently.
  */
@@ -120,7 +121,9 @@ int adamas_encode_keys(const void *K, uint8_t *codes, const int32_t *pos_begin, 
  *   idx       device int32 [B][Hq][budget]  kept token positions in (D, t)
  *                                        order, -1 past k_eff
  *   workspace device, >= adamas_workspace_bytes(...) bytes, zero-filled once
- * The step runs as one cooperative kernel with one block per SM.
+ * The step runs as one kernel launch: one thread-block cluster per (b, kv head),
+ * its blocks splitting the head's tokens and exchanging histograms and partial
+ * softmax states through distributed shared memory.
  */
 int adamas_decode_step(const void *q, const uint8_t *codes, const void *K, const void *V,
                        const int32_t *seq_lens, int B, int Hq, int Hkv, int64_t Nmax, int d,
