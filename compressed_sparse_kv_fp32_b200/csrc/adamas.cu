@@ -342,13 +342,17 @@ static int launch_decode(const DecodeParams& prm, const Plan& P, cudaStream_t st
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = P.smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = (unsigned)P.cluster;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  // the launch may begin while the previous kernel of the stream finishes: the
+  // kernel waits for it (griddepcontrol.wait) before touching global memory
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   const cudaError_t e = P.smem_d ? cudaLaunchKernelEx(&cfg, decode_step_kernel<G, true>, prm)
                                  : cudaLaunchKernelEx(&cfg, decode_step_kernel<G, false>, prm);
   if (e != cudaSuccess) return cuda_fail(e);

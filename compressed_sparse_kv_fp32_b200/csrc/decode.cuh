@@ -207,6 +207,16 @@ __device__ __forceinline__ bool any_le(const uint4 v, uint32_t t1x2) {
   return (a & kHalfTops) != kHalfTops;
 }
 
+// Bit e set when distance e of the eight is <= T; t1x2 = T+1 in both halves.
+__device__ __forceinline__ uint32_t le_bits(const uint4 v, uint32_t t1x2) {
+  const uint32_t l0 = ~((v.x | kHalfTops) - t1x2) & kHalfTops;  // bit 15: low half <= T, bit 31: high half
+  const uint32_t l1 = ~((v.y | kHalfTops) - t1x2) & kHalfTops;
+  const uint32_t l2 = ~((v.z | kHalfTops) - t1x2) & kHalfTops;
+  const uint32_t l3 = ~((v.w | kHalfTops) - t1x2) & kHalfTops;
+  const uint32_t m = (l0 >> 15) | (l1 >> 13) | (l2 >> 11) | (l3 >> 9);  // low halves at 0,2,4,6, high at 16..22
+  return (m | (m >> 15)) & 0xFFu;
+}
+
 // Bit e of lt (eq) set when distance e of the eight is < T (== T); tx2 = T in both
 // halves, t1x2 = T+1 in both halves.
 __device__ __forceinline__ void cand_bits(const uint4 v, uint32_t tx2, uint32_t t1x2, uint32_t& lt, uint32_t& eq) {
@@ -306,6 +316,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const DecodePa
   __shared__ int sm_wmax[kWorkerWarps];
   __shared__ uint32_t sm_acode[kCodeWords];  // the appended key's code
   __shared__ long long sm_tmp[kWorkerWarps];
+  __shared__ uint32_t sm_sink[32];  // per-lane target of the unused atomics of a batch
 
   cg::cluster_group cluster = cg::this_cluster();
   const int C = p.cluster;
@@ -339,6 +350,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const DecodePa
   uint32_t* sm_carry = reinterpret_cast<uint32_t*>(ring + DecodeSmem::cnt());    // [kHistStride]
   int32_t* sm_list = reinterpret_cast<int32_t*>(ring + DecodeSmem::cnt() + DecodeSmem::carry());  // [kListCap]
   int32_t* sm_kept = sm_list + kListCap;                                         // [kKeptCap]
+
+  // The next kernel of the stream may be scheduled at once: it waits here, before
+  // its first global read or write, until the kernels before it are done.
+  grid_launch_dependents();
+  grid_dependency_wait();
 
   // ---- the head's length and this block's tokens (both loads in flight together)
   const int32_t* ap_src = p.append_pos ? p.append_pos + b : p.seq_lens + b;
@@ -381,6 +397,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const DecodePa
   }
   for (int i = tid; i < G * kHistStride; i += kThreads) sm_hist[i] = 0u;
   if (tid < kMaxGroup) sm_T[tid] = kBins - 1;  // always overwritten when the histograms are consistent
+
   __syncthreads();
   // Every block of the cluster has started (and may be written to through
   // distributed shared memory) once every thread has arrived here; each thread
@@ -600,33 +617,51 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const DecodePa
 
       if (grouped) {
         // ---- every token with D <= T to its group (group d at [lpre[d], lpre[d] + hist[d])):
-        // each thread takes a run of 8-position groups, lanes start at different
-        // points of their runs so that a warp's loads spread over the banks
-        const uint32_t tx2 = T | T << 16, t1x2 = (T + 1) | (T + 1) << 16;
+        // each thread takes a run of 8-position groups, eight at a time (lanes start
+        // at different points of the eight so that a warp's loads spread over the
+        // banks), and places its candidates four at a time so that their atomic
+        // cursor updates are in flight together
+        const uint32_t t1x2 = (T + 1) | (T + 1) << 16;
         const int chunk = (ngrp + kWorkers - 1) / kWorkers;
-        const int rot = lane % chunk;
-        for (int k = 0; k < chunk; ++k) {
-          int kk = k + rot;
-          if (kk >= chunk) kk -= chunk;
-          const int grp = tid * chunk + kk;
-          if (grp >= ngrp) continue;
-          const uint4 v = load_dist8<SMEM_D>(drow, grp);
-          if (!any_le(v, t1x2)) continue;
-          uint32_t mlt, meq;
-          cand_bits(v, tx2, t1x2, mlt, meq);
-          for (uint32_t m = mlt | meq; m != 0u; m &= m - 1u) {
-            const int e = __ffs((int)m) - 1;
-            const uint32_t wv = e < 4 ? (e < 2 ? v.x : v.y) : (e < 6 ? v.z : v.w);
-            const uint32_t d = (wv >> (16 * (e & 1))) & 0xFFFFu;
-            const uint32_t c = atomicAdd(&sm_carry[d], 1u);
-            if (c >= hist_g[d]) continue;  // never with consistent histograms (checked below)
-            const uint32_t tpos = (uint32_t)(grp * 8 + e);
-            sm_list[lpre_g[d] + c] = (int32_t)(d << 23 | tpos);
-            const int64_t row = kv_base + t0 + tpos;  // the row is very likely kept: on its way into L2
-            prefetch_l2(p.K + row * kDim);
-            prefetch_l2(p.K + row * kDim + 64);
-            prefetch_l2(p.V + row * kDim);
-            prefetch_l2(p.V + row * kDim + 64);
+        const int rot = lane & 7;
+        for (int k0 = 0; k0 < chunk; k0 += 8) {
+          unsigned long long cm = 0ull;  // bit 8j + e: position (tid * chunk + k0 + j) * 8 + e
+#pragma unroll
+          for (int h = 0; h < 8; h += 2) {
+            uint4 v[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const int j = (h + u + rot) & 7, grp = tid * chunk + k0 + j;
+              v[u] = (k0 + j < chunk && grp < ngrp) ? load_dist8<SMEM_D>(drow, grp)
+                                                    : make_uint4(~0u, ~0u, ~0u, ~0u);
+            }
+#pragma unroll
+            for (int u = 0; u < 2; ++u) cm |= (unsigned long long)le_bits(v[u], t1x2) << (8 * ((h + u + rot) & 7));
+          }
+          while (cm != 0ull) {
+            uint32_t tp[4], dd[4], cc[4];
+            bool ok[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              ok[u] = cm != 0ull;
+              const int bit = ok[u] ? __ffsll((long long)cm) - 1 : 0;
+              cm &= cm - 1ull;
+              tp[u] = ok[u] ? (uint32_t)((tid * chunk + k0 + (bit >> 3)) * 8 + (bit & 7)) : 0u;
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) dd[u] = load_dist1<SMEM_D>(drow, (int)tp[u]);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) cc[u] = atomicAdd(ok[u] ? &sm_carry[dd[u]] : &sm_sink[lane], 1u);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              if (!ok[u] || cc[u] >= hist_g[dd[u]]) continue;  // the latter never with consistent histograms
+              sm_list[lpre_g[dd[u]] + cc[u]] = (int32_t)(dd[u] << 23 | tp[u]);
+              const int64_t row = kv_base + t0 + tp[u];  // the row is very likely kept: on its way into L2
+              prefetch_l2(p.K + row * kDim);
+              prefetch_l2(p.K + row * kDim + 64);
+              prefetch_l2(p.V + row * kDim);
+              prefetch_l2(p.V + row * kDim + 64);
+            }
           }
         }
         worker_sync();
@@ -645,8 +680,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const DecodePa
           const uint32_t e = lds32(smem_addr(sm_list + i));
           const uint32_t d = e >> 23, tpos = e & kPosMask;
           const int gb = (int)lpre_g[d], gn = (int)hist_g[d];
-          int r = 0;
-          for (int q = gb; q < gb + gn; ++q) r += (lds32(smem_addr(sm_list + q)) & kPosMask) < tpos;
+          const int32_t* grp_list = sm_list + gb;  // plain loads: the compiler keeps several in flight
+          int r = 0, q = 0;
+          for (; q + 4 <= gn; q += 4)
+            r += (((uint32_t)grp_list[q] & kPosMask) < tpos) + (((uint32_t)grp_list[q + 1] & kPosMask) < tpos) +
+                 (((uint32_t)grp_list[q + 2] & kPosMask) < tpos) + (((uint32_t)grp_list[q + 3] & kPosMask) < tpos);
+          for (; q < gn; ++q) r += ((uint32_t)grp_list[q] & kPosMask) < tpos;
           const int slot = (int)rank_g[d] + r;
           if (slot < keff) {
             idx_h[slot] = (int32_t)(t0 + tpos);

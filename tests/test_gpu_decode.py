@@ -65,6 +65,9 @@ TINY = [
     (1, 1, 1, 40000, [39999], 3000),
     # distances too many for shared memory: they go through the workspace
     (1, 8, 1, 200000, [200000], 512),
+    # many kept tokens per thread: per-thread phase-1 lists overflow and are rescanned
+    (1, 32, 32, 40000, [40000], 8000),
+    (1, 64, 32, 20000, [20000], 10000),
 ]
 
 
