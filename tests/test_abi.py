@@ -61,6 +61,13 @@ def test_host_side_argument_errors(lib):
     assert lib.adamas_encode_keys(fake, fake, None, -1, 1, 4, 64, 128, None) == -1
     assert lib.adamas_score(fake, fake, fake, 1, 4, 4, 64, 96, fake, None) == -2
     assert lib.adamas_workspace_init(None, 16, None) == -1
+    # fused append step: missing or misaligned positions, and the decode step's own checks
+    assert lib.adamas_decode_step_append(fake, fake, fake, fake, fake, None, 1, 4, 4, 64, 128, 8, fake, fake,
+                                         fake, 1 << 20, None) == -1
+    assert lib.adamas_decode_step_append(fake, fake, fake, fake, fake, P(4098), 1, 4, 4, 64, 128, 8, fake,
+                                         fake, fake, 1 << 20, None) == -1
+    assert lib.adamas_decode_step_append(fake, fake, fake, fake, fake, fake, 1, 4, 4, 64, 64, 8, fake, fake,
+                                         fake, 1 << 20, None) == -2
     # empty batch: nothing to do, nothing touched, no CUDA call
     assert lib.adamas_decode_step(None, None, None, None, None, 0, 4, 4, 64, 128, 8, None, None,
                                   None, 0, None) == 0
