@@ -145,3 +145,45 @@ def decode_step(q, K, V, codes, seq_lens, budget: int, nthreads: int = 1, want_d
                                   nthreads)
     _check(rc, "decode_step")
     return out, idx[:, :, :budget], dist
+
+
+def decode_step_group_shared(q, K, V, codes, seq_lens, budget: int):
+    """Group-shared selection for grouped-query attention (a reading for grouped
+    heads of the ADAMAS article's §2.3 scoring and §5.2 token budget, which the
+    article states per head only): for every (b, kv head) the L1 distances of
+    its G query heads are summed per token, the k_eff = min(budget, len) tokens
+    of smallest (summed distance, index) are kept once, and each query head of
+    the group runs exact attention over those rows.
+
+    q [B,Hq,128], K/V [B,Hkv,Nmax,128] bf16 bits, codes [B,Hkv,Nmax,32] (from
+    encode), seq_lens int32 [B].  Returns (out float64 [B,Hq,128], idx int32
+    [B,Hkv,budget] with -1 past k_eff)."""
+    q = _c(q, np.uint16)
+    K = _c(K, np.uint16)
+    V = _c(V, np.uint16)
+    codes = _c(codes, np.uint8)
+    lens = _c(seq_lens, np.int32)
+    B, Hq, d = q.shape
+    _, Hkv, Nmax, _ = K.shape
+    if Hq % Hkv or V.shape != K.shape or codes.shape != (B, Hkv, Nmax, 32) or lens.shape != (B,):
+        raise ValueError("oracle: inconsistent shapes")
+    G = Hq // Hkv
+    qcodes = encode(q.reshape(-1, d)).reshape(B, Hq, 32)
+    out = np.zeros((B, Hq, d), dtype=np.float64)
+    idx = np.full((B, Hkv, budget), -1, dtype=np.int32)
+    for b in range(B):
+        n = int(lens[b])
+        if n < 0 or n > Nmax:
+            raise ValueError("oracle: sequence length outside [0, Nmax]")
+        keff = min(budget, n)
+        for h in range(Hkv):
+            if keff == 0:
+                continue
+            D = np.zeros(n, dtype=np.int64)
+            for g in range(G):
+                D += distance(qcodes[b, h * G + g], codes[b, h, :n])
+            kept = select(D.astype(np.int32), keff)
+            idx[b, h, :keff] = kept
+            for g in range(G):
+                out[b, h * G + g] = attend(q[b, h * G + g], K[b, h, :n], V[b, h, :n], kept)
+    return out, idx

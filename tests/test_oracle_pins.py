@@ -331,3 +331,73 @@ def test_needles_are_selected_gqa(orc):
             pos = synth.needle_positions(w, b, g, int(inp["lens"][b]))
             for p, h in zip(pos, synth.needle_targets(w, g)):
                 assert p in idx[b, h], (b, g, p, h)
+
+
+# ---- group-shared selection for grouped heads (summed distances, one budget per kv head)
+
+def test_group_shared_with_one_head_per_group_is_the_per_head_step(orc):
+    w = synth.WORKLOADS[2].scaled(Hq=4, Hkv=4, Nmax=300)
+    inp = synth.make_inputs(w)
+    codes = orc.encode(inp["K"])
+    lens = np.array([217], dtype=np.int32)
+    out_s, idx_s = orc.decode_step_group_shared(inp["q"], inp["K"], inp["V"], codes, lens, 40)
+    out_h, idx_h, _ = orc.decode_step(inp["q"], inp["K"], inp["V"], codes, lens, 40)
+    assert np.array_equal(idx_s, idx_h)
+    assert np.abs(out_s - out_h).max() < 1e-12
+
+
+def test_group_shared_matches_brute_force(orc):
+    # distances summed over the group's heads from unpacked 2-bit fields, ranked by
+    # Python's sorted() on (sum, index); attention by torch SDPA over those rows
+    w = synth.WORKLOADS[4].scaled(B=2, Hq=6, Hkv=2, Nmax=48, len_range=None, n_needles=2)
+    inp = synth.make_inputs(w)
+    codes = orc.encode(inp["K"])
+    lens = np.array([48, 29], dtype=np.int32)
+    budget = 11
+    out, idx = orc.decode_step_group_shared(inp["q"], inp["K"], inp["V"], codes, lens, budget)
+    G = 3
+    for b in range(2):
+        n = int(lens[b])
+        for h in range(2):
+            kf = unpack(codes[b, h, :n])
+            total = np.zeros(n, dtype=np.int64)
+            for g in range(G):
+                qf = unpack(orc.encode(inp["q"][b, h * G + g]))
+                total += np.abs(kf - qf).sum(axis=1)
+            want = sorted(range(n), key=lambda t: (total[t], t))[:budget]
+            assert idx[b, h, :len(want)].tolist() == want
+            assert (idx[b, h, len(want):] == -1).all()
+            for g in range(G):
+                ref = _dense_sdpa(inp["q"][b, h * G + g], inp["K"][b, h][want], inp["V"][b, h][want])
+                assert np.abs(out[b, h * G + g] - ref).max() < 1e-12
+
+
+def test_group_shared_with_identical_queries_keeps_the_per_head_rows(orc):
+    # equal query heads: the summed distance is G times each head's, so the order
+    # (and the kept rows) cannot change
+    w = synth.WORKLOADS[4].scaled(B=1, Hq=8, Hkv=2, Nmax=400, len_range=None)
+    inp = synth.make_inputs(w)
+    q = inp["q"].copy()
+    q[:, 1:4] = q[:, 0:1]
+    q[:, 5:8] = q[:, 4:5]
+    codes = orc.encode(inp["K"])
+    lens = np.array([400], dtype=np.int32)
+    out_s, idx_s = orc.decode_step_group_shared(q, inp["K"], inp["V"], codes, lens, 64)
+    out_h, idx_h, _ = orc.decode_step(q, inp["K"], inp["V"], codes, lens, 64)
+    for hq in range(8):
+        assert np.array_equal(idx_s[0, hq // 4], idx_h[0, hq])
+    assert np.abs(out_s - out_h).max() < 1e-12
+
+
+def test_group_shared_budget_and_empty_sequences(orc):
+    w = synth.WORKLOADS[4].scaled(B=2, Hq=4, Hkv=2, Nmax=30, len_range=None)
+    inp = synth.make_inputs(w)
+    codes = orc.encode(inp["K"])
+    lens = np.array([0, 30], dtype=np.int32)
+    out, idx = orc.decode_step_group_shared(inp["q"], inp["K"], inp["V"], codes, lens, 50)
+    assert (idx[0] == -1).all() and (out[0] == 0).all()
+    for h in range(2):
+        assert sorted(idx[1, h, :30].tolist()) == list(range(30)) and (idx[1, h, 30:] == -1).all()
+        for g in range(2):  # budget >= len: dense attention over the whole sequence
+            ref = _dense_sdpa(inp["q"][1, 2 * h + g], inp["K"][1, h], inp["V"][1, h])
+            assert np.abs(out[1, 2 * h + g] - ref).max() < 1e-12
