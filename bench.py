@@ -294,28 +294,32 @@ def run_gpu(args, rank, world):
 
     # ---- end to end through the Python API: pinned host inputs in, results out, every step
     e2e_steps = min(args.e2e_steps, K_steps)
-    q_pin = torch.from_numpy(synth.query(w, 3).view(np.int16)).view(torch.bfloat16).pin_memory()
-    krow_pin = torch.from_numpy(K_host[:, :, ctx - 1].copy().view(np.int16)).view(torch.bfloat16).pin_memory()
-    vrow_pin = torch.from_numpy(V_host[:, :, ctx - 1].copy().view(np.int16)).view(torch.bfloat16).pin_memory()
-    out_pin = torch.empty((B, Hq, d), dtype=torch.float32).pin_memory()
-    idx_pin = torch.empty((B, Hq, BUDGET), dtype=torch.int32).pin_memory()
-    q_dev = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=dev)
-    krow_dev = torch.empty((B, Hkv, d), dtype=torch.bfloat16, device=dev)
-    vrow_dev = torch.empty_like(krow_dev)
-    h2d = q_pin.numel() * 2 + krow_pin.numel() * 2 + vrow_pin.numel() * 2
-    d2h = out_pin.numel() * 4 + idx_pin.numel() * 4
+    # the step's inputs (q, new K row, new V row) travel in one pinned buffer and
+    # its results (out, idx) come back in one: one copy each way per step
+    nq, nkv = B * Hq * d, B * Hkv * d
+    in_pin = torch.empty(nq + 2 * nkv, dtype=torch.bfloat16).pin_memory()
+    in_pin[:nq].copy_(torch.from_numpy(synth.query(w, 3).reshape(-1).view(np.int16)).view(torch.bfloat16))
+    in_pin[nq:nq + nkv].copy_(torch.from_numpy(K_host[:, :, ctx - 1].reshape(-1).view(np.int16)).view(torch.bfloat16))
+    in_pin[nq + nkv:].copy_(torch.from_numpy(V_host[:, :, ctx - 1].reshape(-1).view(np.int16)).view(torch.bfloat16))
+    in_dev = torch.empty_like(in_pin, device=dev)
+    q_dev = in_dev[:nq].view(B, Hq, d)
+    krow_dev = in_dev[nq:nq + nkv].view(B, Hkv, d)
+    vrow_dev = in_dev[nq + nkv:].view(B, Hkv, d)
+    n_out, n_idx = B * Hq * d, B * Hq * BUDGET   # fp32 and int32 words
+    res_dev = torch.empty(n_out + n_idx, dtype=torch.int32, device=dev)
+    res_pin = torch.empty_like(res_dev, device="cpu").pin_memory()
+    out_dev = res_dev[:n_out].view(torch.float32).view(B, Hq, d)
+    idx_dev = res_dev[n_out:].view(B, Hq, BUDGET)
+    h2d = in_pin.numel() * 2
+    d2h = res_pin.numel() * 4
 
     def e2e_step(i):
         L = layers[i % n_layers]
-        q_dev.copy_(q_pin, non_blocking=True)
-        krow_dev.copy_(krow_pin, non_blocking=True)
-        vrow_dev.copy_(vrow_pin, non_blocking=True)
+        in_dev.copy_(in_pin, non_blocking=True)
         L["K"][:, :, ctx - 1].copy_(krow_dev)
         L["V"][:, :, ctx - 1].copy_(vrow_dev)
-        adamas.decode_step_append(q_dev, L["codes"], L["K"], L["V"], lens, pos, BUDGET, L["ws"], L["out"],
-                                  L["idx"])
-        out_pin.copy_(L["out"], non_blocking=True)
-        idx_pin.copy_(L["idx"], non_blocking=True)
+        adamas.decode_step_append(q_dev, L["codes"], L["K"], L["V"], lens, pos, BUDGET, L["ws"], out_dev, idx_dev)
+        res_pin.copy_(res_dev, non_blocking=True)
         torch.cuda.current_stream().synchronize()
 
     for i in range(3 if e2e_steps > 0 else 0):
