@@ -187,3 +187,48 @@ def decode_step_group_shared(q, K, V, codes, seq_lens, budget: int):
             for g in range(G):
                 out[b, h * G + g] = attend(q[b, h * G + g], K[b, h, :n], V[b, h, :n], kept)
     return out, idx
+
+
+def decode_step_forced(q, K, V, codes, seq_lens, budget: int, n_sink: int, n_recent: int):
+    """Per-head decode step with forced rows: the first n_sink tokens (attention
+    sinks) and the last n_recent tokens of each sequence (the recent window)
+    rank ahead of every scored token, as if their distance were -1; the rest is
+    the per-head step (k_eff = min(budget, len) tokens of smallest (D, index)).
+    Forced rows therefore come first in idx, in index order, and when there are
+    more of them than k_eff the lowest indices win.  (A reading of the ADAMAS
+    article's §3.2 / §6 tuning advice -- some tokens keep full attention -- for
+    the sink and window the other pages describe; the article gives no rule.)
+
+    Shapes as decode_step.  Returns (out float64 [B,Hq,128], idx int32 [B,Hq,budget])."""
+    q = _c(q, np.uint16)
+    K = _c(K, np.uint16)
+    V = _c(V, np.uint16)
+    codes = _c(codes, np.uint8)
+    lens = _c(seq_lens, np.int32)
+    B, Hq, d = q.shape
+    _, Hkv, Nmax, _ = K.shape
+    if Hq % Hkv or V.shape != K.shape or codes.shape != (B, Hkv, Nmax, 32) or lens.shape != (B,):
+        raise ValueError("oracle: inconsistent shapes")
+    if n_sink < 0 or n_recent < 0:
+        raise ValueError("oracle: negative forced-row counts")
+    G = Hq // Hkv
+    qcodes = encode(q.reshape(-1, d)).reshape(B, Hq, 32)
+    out = np.zeros((B, Hq, d), dtype=np.float64)
+    idx = np.full((B, Hq, budget), -1, dtype=np.int32)
+    for b in range(B):
+        n = int(lens[b])
+        if n < 0 or n > Nmax:
+            raise ValueError("oracle: sequence length outside [0, Nmax]")
+        keff = min(budget, n)
+        if keff == 0:
+            continue
+        t = np.arange(n)
+        forced = (t < n_sink) | (t >= n - n_recent)
+        for hq in range(Hq):
+            h = hq // G
+            D = distance(qcodes[b, hq], codes[b, h, :n])
+            D[forced] = -1
+            kept = select(D, keff)
+            idx[b, hq, :keff] = kept
+            out[b, hq] = attend(q[b, hq], K[b, h, :n], V[b, h, :n], kept)
+    return out, idx

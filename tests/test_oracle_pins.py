@@ -401,3 +401,48 @@ def test_group_shared_budget_and_empty_sequences(orc):
         for g in range(2):  # budget >= len: dense attention over the whole sequence
             ref = _dense_sdpa(inp["q"][1, 2 * h + g], inp["K"][1, h], inp["V"][1, h])
             assert np.abs(out[1, 2 * h + g] - ref).max() < 1e-12
+
+
+# ---- forced rows (attention sinks and the recent window rank ahead of scored tokens)
+
+def test_forced_rows_none_is_the_plain_step(orc):
+    w = synth.WORKLOADS[4].scaled(B=2, Hq=4, Hkv=2, Nmax=200, len_range=(90, 200))
+    inp = synth.make_inputs(w)
+    codes = orc.encode(inp["K"])
+    out_f, idx_f = orc.decode_step_forced(inp["q"], inp["K"], inp["V"], codes, inp["lens"], 24, 0, 0)
+    out_p, idx_p, _ = orc.decode_step(inp["q"], inp["K"], inp["V"], codes, inp["lens"], 24)
+    assert np.array_equal(idx_f, idx_p)
+    assert np.abs(out_f - out_p).max() < 1e-12
+
+
+def test_forced_rows_match_brute_force(orc):
+    w = synth.WORKLOADS[4].scaled(B=2, Hq=4, Hkv=2, Nmax=40, len_range=None, n_needles=2)
+    inp = synth.make_inputs(w)
+    codes = orc.encode(inp["K"])
+    lens = np.array([40, 13], dtype=np.int32)
+    n_sink, n_recent = 3, 5
+    for budget in (4, 10, 20):  # fewer, as many as and more than the forced rows
+        out, idx = orc.decode_step_forced(inp["q"], inp["K"], inp["V"], codes, lens, budget, n_sink, n_recent)
+        for b in range(2):
+            n = int(lens[b])
+            for hq in range(4):
+                h = hq // 2
+                D = np.abs(unpack(codes[b, h, :n]) - unpack(orc.encode(inp["q"][b, hq]))).sum(axis=1)
+                rank = [(-1 if (t < n_sink or t >= n - n_recent) else int(D[t]), t) for t in range(n)]
+                want = [t for _, t in sorted(rank)][:min(budget, n)]
+                assert idx[b, hq, :len(want)].tolist() == want
+                assert (idx[b, hq, len(want):] == -1).all()
+                ref = _dense_sdpa(inp["q"][b, hq], inp["K"][b, h][want], inp["V"][b, h][want])
+                assert np.abs(out[b, hq] - ref).max() < 1e-12
+
+
+def test_forced_rows_are_always_kept_when_they_fit(orc):
+    w = synth.WORKLOADS[2].scaled(Hq=2, Hkv=2, Nmax=1000)
+    inp = synth.make_inputs(w)
+    codes = orc.encode(inp["K"])
+    lens = np.array([1000], dtype=np.int32)
+    _, idx = orc.decode_step_forced(inp["q"], inp["K"], inp["V"], codes, lens, 64, 4, 16)
+    forced = list(range(4)) + list(range(984, 1000))
+    for hq in range(2):
+        assert idx[0, hq, :20].tolist() == forced
+        assert len(set(idx[0, hq].tolist())) == 64
