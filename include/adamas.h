@@ -123,7 +123,11 @@ int adamas_encode_keys(const void *K, uint8_t *codes, const int32_t *pos_begin, 
  *   workspace device, >= adamas_workspace_bytes(...) bytes, zero-filled once
  * The step runs as one kernel launch: one thread-block cluster per (b, kv head),
  * its blocks splitting the head's tokens and exchanging histograms and partial
- * softmax states through distributed shared memory.
+ * softmax states through distributed shared memory.  The launch opts in to
+ * programmatic dependent launch: its blocks may be scheduled while the previous
+ * kernel of the stream drains, and each waits for that kernel to complete (and
+ * its writes to be visible) before its first global read or write, so stream
+ * order semantics are unchanged.
  */
 int adamas_decode_step(const void *q, const uint8_t *codes, const void *K, const void *V,
                        const int32_t *seq_lens, int B, int Hq, int Hkv, int64_t Nmax, int d,
