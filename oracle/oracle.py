@@ -232,3 +232,38 @@ def decode_step_forced(q, K, V, codes, seq_lens, budget: int, n_sink: int, n_rec
             idx[b, hq, :keff] = kept
             out[b, hq] = attend(q[b, hq], K[b, h, :n], V[b, h, :n], kept)
     return out, idx
+
+
+def decode_step_paged(q, K_pages, V_pages, code_pages, block_table, seq_lens, budget: int):
+    """Per-head decode step over a paged cache: token t of sequence b lives in
+    physical page block_table[b, t // P] at offset t % P (P = page size, the
+    pages' second dimension).  K_pages/V_pages [n_pages, P, Hkv, 128] bf16 bits,
+    code_pages [n_pages, P, Hkv, 32], block_table int32 [B, max_pages].  The
+    tokens are read through the table into sequence order and the plain step
+    runs on them.  Returns (out float64 [B,Hq,128], idx int32 [B,Hq,budget])."""
+    K_pages = _c(K_pages, np.uint16)
+    V_pages = _c(V_pages, np.uint16)
+    code_pages = _c(code_pages, np.uint8)
+    table = _c(block_table, np.int32)
+    lens = _c(seq_lens, np.int32)
+    n_pages, P, Hkv, d = K_pages.shape
+    B, max_pages = table.shape
+    if V_pages.shape != K_pages.shape or code_pages.shape != (n_pages, P, Hkv, 32) or lens.shape != (B,):
+        raise ValueError("oracle: inconsistent shapes")
+    Nmax = max_pages * P
+    K = np.zeros((B, Hkv, Nmax, d), dtype=np.uint16)
+    V = np.zeros_like(K)
+    codes = np.zeros((B, Hkv, Nmax, 32), dtype=np.uint8)
+    for b in range(B):
+        n = int(lens[b])
+        if n < 0 or n > Nmax:
+            raise ValueError("oracle: sequence length outside the table")
+        for t in range(n):
+            page = int(table[b, t // P])
+            if not 0 <= page < n_pages:
+                raise ValueError("oracle: block table entry out of range")
+            K[b, :, t] = K_pages[page, t % P]
+            V[b, :, t] = V_pages[page, t % P]
+            codes[b, :, t] = code_pages[page, t % P]
+    out, idx, _ = decode_step(q, K, V, codes, lens, budget)
+    return out, idx

@@ -446,3 +446,41 @@ def test_forced_rows_are_always_kept_when_they_fit(orc):
     for hq in range(2):
         assert idx[0, hq, :20].tolist() == forced
         assert len(set(idx[0, hq].tolist())) == 64
+
+
+# ---- paged cache (a block table maps each sequence's logical pages to physical pages)
+
+def test_paged_step_equals_the_contiguous_step(orc):
+    # scatter a contiguous cache into shuffled physical pages; reading through the
+    # table must give the contiguous step back exactly
+    w = synth.WORKLOADS[4].scaled(B=3, Hq=4, Hkv=2, Nmax=96, len_range=None, n_needles=2)
+    inp = synth.make_inputs(w)
+    codes = orc.encode(inp["K"])
+    lens = np.array([96, 37, 1], dtype=np.int32)
+    P, max_pages = 16, 6
+    rng = np.random.default_rng(5)
+    n_pages = 3 * max_pages + 4
+    perm = rng.permutation(n_pages)[:3 * max_pages].reshape(3, max_pages).astype(np.int32)
+    Kp = rng.integers(0, 2 ** 16, size=(n_pages, P, 2, 128), dtype=np.uint16)  # garbage where unused
+    Vp = rng.integers(0, 2 ** 16, size=(n_pages, P, 2, 128), dtype=np.uint16) & np.uint16(0x3FFF)
+    Kp &= np.uint16(0x3FFF)
+    Cp = rng.integers(0, 256, size=(n_pages, P, 2, 32), dtype=np.uint8)
+    for b in range(3):
+        for lp in range(max_pages):
+            page = perm[b, lp]
+            Kp[page] = inp["K"][b, :, lp * P:(lp + 1) * P].transpose(1, 0, 2)
+            Vp[page] = inp["V"][b, :, lp * P:(lp + 1) * P].transpose(1, 0, 2)
+            Cp[page] = codes[b, :, lp * P:(lp + 1) * P].transpose(1, 0, 2)
+    out_p, idx_p = orc.decode_step_paged(inp["q"], Kp, Vp, Cp, perm, lens, 20)
+    out_c, idx_c, _ = orc.decode_step(inp["q"], inp["K"], inp["V"], codes, lens, 20)
+    assert np.array_equal(idx_p, idx_c)
+    assert np.array_equal(out_p, out_c)
+
+
+def test_paged_step_rejects_a_bad_table(orc):
+    w = synth.WORKLOADS[2].scaled(Hq=2, Hkv=2, Nmax=32)
+    inp = synth.make_inputs(w)
+    Kp = np.zeros((2, 16, 2, 128), np.uint16)
+    Cp = np.zeros((2, 16, 2, 32), np.uint8)
+    with pytest.raises(ValueError):
+        orc.decode_step_paged(inp["q"], Kp, Kp, Cp, np.array([[0, 5]], np.int32), np.array([32], np.int32), 4)
