@@ -103,6 +103,46 @@ def test_rotation_preserves_inner_products(orc):
     assert (np.abs(lhs - rhs) <= bound).all()
 
 
+def _butterfly_f32(x_bits, widths):
+    """NumPy float32 restatement of the rotation: one elementwise add/subtract per
+    butterfly stage over the whole batch, stage widths in the given order, then one
+    multiply by C (NumPy float32 arithmetic rounds to nearest and never fuses)."""
+    y = synth.bf16_to_f32(x_bits).astype(np.float32).copy()
+    idx = np.arange(128)
+    for h in widths:
+        lo = idx[(idx & h) == 0]
+        a, b = y[:, lo].copy(), y[:, lo + h].copy()
+        y[:, lo] = a + b
+        y[:, lo + h] = a - b
+    return y * C
+
+
+def _codes_f32(y):
+    """Bucketing and MSB-first packing of float32 rotated rows, restated in NumPy."""
+    m = np.abs(y).max(1, keepdims=True)
+    c = (3 - (y < -0.5 * m).astype(np.int64) - (y < 0).astype(np.int64)
+         - (y < 0.5 * m).astype(np.int64)).reshape(y.shape[0], 32, 4)
+    return (c[..., 0] << 6 | c[..., 1] << 4 | c[..., 2] << 2 | c[..., 3]).astype(np.uint8)
+
+
+def test_rotation_stage_order_is_ascending_bit_for_bit(orc):
+    # The fp32 rounding sequence is part of the contract (codes are reproducible bit for
+    # bit): widths 1, 2, ..., 64 ascending, no fused multiply-add, one final multiply by C.
+    # Bounds alone cannot see the stage order, so an independent float32 restatement must
+    # agree on every bit of every rotated value and every code byte, and the reversed
+    # order must give other bits on many vectors, which shows that this check can tell
+    # the orders apart (codes move only where a value lands on a threshold, so they
+    # rarely differ).
+    x = np.concatenate([random_vectors(10000, 21), random_vectors(10000, 22, outliers=False)])
+    want = _butterfly_f32(x, [1, 2, 4, 8, 16, 32, 64])
+    got = orc.rotate(x)
+    assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
+    assert np.array_equal(orc.encode(x), _codes_f32(want))
+    rev = _butterfly_f32(x, [64, 32, 16, 8, 4, 2, 1])
+    differ = (rev.view(np.uint32) != got.view(np.uint32)).any(axis=1)
+    assert differ.sum() > 100
+
+
 def test_rotation_spreads_outliers(orc):
     # qualitative claim of §2.1: the rotation flattens outlier channels
     x = random_vectors(1000, 4)
