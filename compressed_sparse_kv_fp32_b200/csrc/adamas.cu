@@ -19,50 +19,116 @@
 namespace adamas {
 
 // ------------------------------------------------------------------ key encoder
-constexpr int kEncThreads = 128;       // one vector per thread, one tile of 128 positions per block
-constexpr int kEncRowWords = 68;       // 64 words of bf16 + 4 words of padding (bank spread)
+// Prefill: one vector per thread.  Work is handed out in tiles of 32 consecutive
+// positions of one (b, kv head), one tile per warp at a time: the warp copies the
+// next tile into its other shared-memory buffer with coalesced 16-byte cp.async
+// (two rows per instruction) while it encodes the current one, each lane reading
+// its own row.  Rows are padded to 272 B, so the 16-byte reads of a quarter-warp
+// fall into distinct banks.  The loop has no block-wide barrier.
+constexpr int kEncWarps = 4;
+constexpr int kEncThreads = 32 * kEncWarps;
+constexpr int kEncRowBytes = 272;
+constexpr int kEncWarpStage = 32 * kEncRowBytes;
+constexpr size_t kEncSmem = (size_t)2 * kEncWarps * kEncWarpStage;  // 69,632 B
+constexpr int kEncBlocksPerSm = 3;
 
-__global__ void __launch_bounds__(kEncThreads) encode_keys_kernel(const uint16_t* __restrict__ K,
-                                                                  uint8_t* __restrict__ codes,
-                                                                  const int32_t* __restrict__ pos_begin,
-                                                                  int count, int Hkv, int64_t Nmax) {
-  __shared__ __align__(16) uint32_t tile[kEncThreads * kEncRowWords];
-  const int tid = threadIdx.x;
-  const int hk = blockIdx.y;
-  const int b = hk / Hkv;
-  const int64_t p0 = pos_begin ? (int64_t)pos_begin[b] : 0;
-  const int64_t first = (int64_t)blockIdx.x * kEncThreads;
-  const uint16_t* kbase = K + (int64_t)hk * Nmax * kDim;
+__global__ void __launch_bounds__(kEncThreads, kEncBlocksPerSm)
+    encode_keys_kernel(const uint16_t* __restrict__ K, uint8_t* __restrict__ codes,
+                       const int32_t* __restrict__ pos_begin, int count, int Hkv, int64_t Nmax, int tiles_per_head,
+                       int heads) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  unsigned char* wbuf = smem + (size_t)warp * 2 * kEncWarpStage;
 
-  // coalesced 16-byte loads of the tile's rows into padded shared memory
-#pragma unroll 4
-  for (int i = tid; i < kEncThreads * 16; i += kEncThreads) {
-    const int row = i >> 4, ch = i & 15;
-    const int64_t r = first + row, pos = p0 + r;
-    if (r < count && pos >= 0 && pos < Nmax) {
-      const uint4 v = *reinterpret_cast<const uint4*>(kbase + pos * kDim + ch * 8);
-      *reinterpret_cast<uint4*>(&tile[row * kEncRowWords + ch * 4]) = v;
-    }
-  }
-  __syncthreads();
+  // The warp's tiles are T = first + k * nwarps; T = hk * tiles_per_head + tin.  The
+  // walk is kept incremental (one division per warp) so that the per-tile cost stays
+  // a few integer operations.
+  const int nwarps = gridDim.x * kEncWarps;
+  const int first = blockIdx.x * kEncWarps + warp;
+  int hk = first / tiles_per_head, tin = first - hk * tiles_per_head;
+  const int dhk = nwarps / tiles_per_head, dtin = nwarps - dhk * tiles_per_head;
 
-  const int64_t r = first + tid, pos = p0 + r;
-  if (r >= count || pos < 0 || pos >= Nmax) return;
-  float v[kDim];
+  // the tile (hk, tin): positions p0 + [0, 32) of head hk, rows [lo, hi) of it valid
+  struct Tile {
+    const uint16_t* src;  // key row of offset 0
+    uint8_t* dst;         // code row of offset 0
+    int lo, hi;
+  };
+  auto tile_of = [&](int h, int t) {
+    const int off0 = t * 32;
+    const int64_t p0 = (pos_begin ? (int64_t)pos_begin[(unsigned)h / (unsigned)Hkv] : 0) + off0;
+    const int64_t row0 = (int64_t)h * Nmax + p0;
+    const int64_t lo = p0 < 0 ? -p0 : 0;
+    int64_t hi = count - off0 < 32 ? count - off0 : 32;
+    if (Nmax - p0 < hi) hi = Nmax - p0;
+    Tile r;
+    r.src = K + row0 * kDim;
+    r.dst = codes + row0 * kCodeBytes;
+    r.lo = (int)(lo < 32 ? lo : 32);
+    r.hi = (int)(hi < r.lo ? r.lo : hi);
+    return r;
+  };
+  auto issue = [&](const Tile& t, int stage) {
+    // lane l copies 16-byte chunk (l mod 16) of rows 2 s + l / 16
+    unsigned char* dst = wbuf + (size_t)stage * kEncWarpStage + (lane >> 4) * kEncRowBytes + (lane & 15) * 16;
+    const uint16_t* src = t.src + (lane >> 4) * kDim + (lane & 15) * 8;
+    if (t.lo == 0 && t.hi == 32) {  // a whole tile: constant offsets, no checks
 #pragma unroll
-  for (int ch = 0; ch < 16; ++ch) {
-    const uint4 w = *reinterpret_cast<const uint4*>(&tile[tid * kEncRowWords + ch * 4]);
-    v[8 * ch + 0] = bf16_lo(w.x); v[8 * ch + 1] = bf16_hi(w.x);
-    v[8 * ch + 2] = bf16_lo(w.y); v[8 * ch + 3] = bf16_hi(w.y);
-    v[8 * ch + 4] = bf16_lo(w.z); v[8 * ch + 5] = bf16_hi(w.z);
-    v[8 * ch + 6] = bf16_lo(w.w); v[8 * ch + 7] = bf16_hi(w.w);
+      for (int s = 0; s < 16; ++s) cp_async16(dst + 2 * s * kEncRowBytes, src + 2 * s * kDim);
+    } else {
+#pragma unroll
+      for (int s = 0; s < 16; ++s) {
+        const int r = 2 * s + (lane >> 4);
+        if (r >= t.lo && r < t.hi) cp_async16(dst + 2 * s * kEncRowBytes, src + 2 * s * kDim);
+      }
+    }
+    cp_async_commit();
+  };
+
+  bool more = hk < heads;
+  Tile cur = tile_of(more ? hk : 0, more ? tin : 0);
+  if (more) issue(cur, 0);
+  else cp_async_commit();
+  for (int k = 0; more; ++k) {
+    tin += dtin;
+    hk += dhk;
+    if (tin >= tiles_per_head) {
+      tin -= tiles_per_head;
+      ++hk;
+    }
+    more = hk < heads;
+    Tile nxt = cur;
+    if (more) {
+      nxt = tile_of(hk, tin);
+      issue(nxt, (k + 1) & 1);
+    } else {
+      cp_async_commit();
+    }
+    cp_async_wait<1>();  // this lane's copies of the current tile have landed
+    __syncwarp();        // ... and every other lane's
+    const bool ok = lane >= cur.lo && lane < cur.hi;
+    uint64_t P[kDim / 2];
+    const unsigned char* row = wbuf + (size_t)(k & 1) * kEncWarpStage + lane * kEncRowBytes;
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+      const uint4 v = ok ? *reinterpret_cast<const uint4*>(row + c * 16) : make_uint4(0u, 0u, 0u, 0u);
+      P[4 * c + 0] = rotate_pair_first(v.x);
+      P[4 * c + 1] = rotate_pair_first(v.y);
+      P[4 * c + 2] = rotate_pair_first(v.z);
+      P[4 * c + 3] = rotate_pair_first(v.w);
+    }
+    __syncwarp();  // every lane has read its row before the buffer is refilled
+    if (ok) {
+      rotate_pairs_rest(P);
+      uint32_t w[kCodeWords];
+      bucket_pack_pairs(P, w);
+      uint4* dst = reinterpret_cast<uint4*>(cur.dst + lane * kCodeBytes);
+      dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+      dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+    }
+    cur = nxt;
   }
-  fwht128_thread(v);
-  uint32_t w[kCodeWords];
-  bucket_pack_thread(v, w);
-  uint4* dst = reinterpret_cast<uint4*>(codes + ((int64_t)hk * Nmax + pos) * kCodeBytes);
-  dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-  dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+  cp_async_wait<0>();
 }
 
 // Small encodes (appending a few tokens): one warp per vector, so a call costs
@@ -150,6 +216,7 @@ struct DeviceInfo {
   bool attrs_set[2][kMaxGroup + 1] = {};
   OccEntry occ[kOccCache] = {};
   int n_occ = 0;
+  int enc_blocks_per_sm = 0;  // resident prefill-encoder blocks per SM (0: not yet set up)
 };
 
 static std::mutex g_mutex;
@@ -194,6 +261,20 @@ static int kernel_attrs(DeviceInfo& dev, const void* fn, int G, bool smem_d) {
   if (e == cudaSuccess) e = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   if (e != cudaSuccess) return cuda_fail(e);
   dev.attrs_set[smem_d ? 1 : 0][G] = true;
+  return ADAMAS_OK;
+}
+
+// One-time set-up of the prefill encoder on a device: its dynamic shared memory
+// and how many of its blocks an SM holds (the persistent grid's size).
+static int encoder_attrs(DeviceInfo& dev) {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (dev.enc_blocks_per_sm > 0) return ADAMAS_OK;
+  const void* fn = reinterpret_cast<const void*>(&encode_keys_kernel);
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kEncSmem);
+  int n = 0;
+  if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, kEncThreads, kEncSmem);
+  if (e != cudaSuccess) return cuda_fail(e);
+  dev.enc_blocks_per_sm = n < 1 ? 1 : n;
   return ADAMAS_OK;
 }
 
@@ -473,7 +554,6 @@ int adamas_encode_keys(const void* K, uint8_t* codes, const int32_t* pos_begin, 
   if (B == 0 || count == 0 || Nmax == 0) return ADAMAS_OK;
   if (!K || !codes || !aligned(K, 16) || !aligned(codes, 32)) return ADAMAS_ERR_INVALID_ARG;
   if (pos_begin && !aligned(pos_begin, 4)) return ADAMAS_ERR_INVALID_ARG;
-  const dim3 grid((unsigned)((count + kEncThreads - 1) / kEncThreads), (unsigned)(B * Hkv));
   const int64_t nvec = (int64_t)count * B * Hkv;
   if (nvec <= kEncWarpMaxVectors) {
     const int per_block = kEncWarpThreads / 32;
@@ -481,8 +561,18 @@ int adamas_encode_keys(const void* K, uint8_t* codes, const int32_t* pos_begin, 
                               (cudaStream_t)stream>>>(static_cast<const uint16_t*>(K), codes, pos_begin, count, Hkv,
                                                       Nmax, nvec);
   } else {
-    encode_keys_kernel<<<grid, kEncThreads, 0, (cudaStream_t)stream>>>(
-        static_cast<const uint16_t*>(K), codes, pos_begin, count, Hkv, Nmax);
+    DeviceInfo* dev = nullptr;
+    int rc2 = device_info(&dev);
+    if (rc2 != ADAMAS_OK) return rc2;
+    if ((rc2 = encoder_attrs(*dev)) != ADAMAS_OK) return rc2;
+    const int tiles_per_head = (int)(((int64_t)count + 31) / 32);
+    const int64_t ntiles = (int64_t)tiles_per_head * B * Hkv;
+    if (ntiles > INT32_MAX) return ADAMAS_ERR_UNSUPPORTED;
+    const int64_t want = (ntiles + kEncWarps - 1) / kEncWarps;
+    const int64_t cap = (int64_t)dev->sms * dev->enc_blocks_per_sm;
+    const unsigned grid = (unsigned)(want < cap ? want : cap);
+    encode_keys_kernel<<<grid, kEncThreads, kEncSmem, (cudaStream_t)stream>>>(
+        static_cast<const uint16_t*>(K), codes, pos_begin, count, Hkv, Nmax, tiles_per_head, B * Hkv);
   }
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);

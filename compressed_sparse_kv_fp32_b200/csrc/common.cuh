@@ -32,18 +32,6 @@ __device__ __forceinline__ void ld_stream_v8(const void* p, uint32_t (&r)[8]) {
                : "l"(p));
 }
 
-__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
-  uint32_t v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-
-__device__ __forceinline__ unsigned long long ld_acquire_gpu64(const unsigned long long* p) {
-  unsigned long long v;
-  asm volatile("ld.acquire.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-  return v;
-}
-
 // ---------------------------------------------------------------- bulk async copies (no multicast)
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(p);
@@ -59,18 +47,6 @@ __device__ __forceinline__ uint4 lds128(uint32_t a) {
 __device__ __forceinline__ uint32_t lds32(uint32_t a) {
   uint32_t v;
   asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
-  return v;
-}
-// Shared-window address of the same location in cluster block `rank`, and a
-// relaxed cluster-scope load from such an address (several may be in flight).
-__device__ __forceinline__ uint32_t mapa_shared(uint32_t a, int rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
-  return r;
-}
-__device__ __forceinline__ uint32_t ld_relaxed_cluster(uint32_t a) {
-  uint32_t v;
-  asm volatile("ld.relaxed.cluster.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
   return v;
 }
 // Split cluster barrier: arrive (release: this thread's earlier writes become
@@ -105,30 +81,18 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
 }
 
 // One global -> shared bulk copy (16-byte aligned addresses, size a multiple of 16)
-// whose completion is counted in bytes on `bar`.
+// whose completion is counted in bytes on `bar`.  The source is read once, so its
+// lines are marked first to go from L2 (they should not push out data that is read
+// again, like the K/V rows of the gather).
 __device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+      "{\n .reg .b64 pol;\n createpolicy.fractional.L2::evict_first.b64 pol, 1.0;\n"
+      " cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], pol;\n}" ::"r"(
           smem_addr(dst)),
       "l"(src), "r"(bytes), "r"(smem_addr(bar))
       : "memory");
 }
 
-__device__ __forceinline__ unsigned long long ld_relaxed_gpu64(const unsigned long long* p) {
-  unsigned long long v;
-  asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-  return v;
-}
-
-__device__ __forceinline__ unsigned long long atom_add_acqrel_gpu64(unsigned long long* p, unsigned long long v) {
-  unsigned long long old;
-  asm volatile("atom.acq_rel.gpu.global.add.u64 %0, [%1], %2;" : "=l"(old) : "l"(p), "l"(v) : "memory");
-  return old;
-}
-
-__device__ __forceinline__ void red_add_release_gpu64(unsigned long long* p, unsigned long long v) {
-  asm volatile("red.release.gpu.global.add.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
 
 // 16-byte global -> shared copy through the L2 (cp.async, completion by wait_group).
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
@@ -145,11 +109,6 @@ __device__ __forceinline__ void prefetch_l2(const void* p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(p) : "memory");
 }
 
-// Bring the 128-byte line holding `p` into L2, to be kept there preferentially.
-__device__ __forceinline__ void prefetch_l2_keep(const void* p) {
-  asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(p) : "memory");
-}
-
 // Bounded wait for the phase with the given parity of `bar` to complete.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t limit) {
   const uint32_t a = smem_addr(bar);
@@ -163,29 +122,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
     if (done) return true;
   }
   return false;
-}
-
-__device__ __forceinline__ uint32_t lop3_xor_and(uint32_t a, uint32_t b, uint32_t c) {
-  // (a ^ b) & c
-  uint32_t r;
-  asm("lop3.b32 %0, %1, %2, %3, 0x28;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
-  return r;
-}
-
-__device__ __forceinline__ uint32_t lop3_xor_andnot(uint32_t a, uint32_t b, uint32_t c) {
-  // (a ^ b) & ~c
-  uint32_t r;
-  asm("lop3.b32 %0, %1, %2, %3, 0x14;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
-  return r;
-}
-
-// Unit x of a range [0, total) split evenly over S blocks: block s owns
-// [s*total/S, (s+1)*total/S).  Returns the owner of x (0 <= x < total).
-__device__ __forceinline__ int owner_of(int64_t x, int64_t total, int S) {
-  return (int)(((x + 1) * (int64_t)S - 1) / total);
-}
-__device__ __forceinline__ int64_t range_begin(int s, int64_t total, int S) {
-  return ((int64_t)s * total) / S;
 }
 
 }  // namespace adamas

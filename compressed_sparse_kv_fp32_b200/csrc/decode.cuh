@@ -167,16 +167,6 @@ __device__ __forceinline__ long long worker_exclusive_scan(long long v, long lon
   return before + x - v;
 }
 
-// Inclusive warp scan.
-__device__ __forceinline__ int warp_inclusive_scan(int x, int lane) {
-#pragma unroll
-  for (int o = 1; o < 32; o *= 2) {
-    const int y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
-  return x;
-}
-
 // Eight consecutive distances 8*grp .. 8*grp+7 as four words of u16 pairs (element
 // 2j in the low half of word j); SMEM: the row is in shared memory.
 template <bool SMEM>
@@ -852,18 +842,31 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const DecodePa
       }
       // ---- half-warp states -> this block's partial state -> the head's owner
       {
-        float* st = sm_state + hw * kPartial;
-        if (hl == 0) { st[0] = m_run; st[1] = l_run; }
+        // the two half-warps of a warp hold the same slice of dimensions: merge them
+        // with shuffles first, then one state per warp goes through shared memory
+        const float m_o = __shfl_xor_sync(0xffffffffu, m_run, 16);
+        const float l_o = __shfl_xor_sync(0xffffffffu, l_run, 16);
+        const float m_new = fmaxf(m_run, m_o);
+        const float a = m_run == -INFINITY ? 0.0f : exp2f(m_run - m_new);  // 0 for a half-warp without rows
+        const float a_o = m_o == -INFINITY ? 0.0f : exp2f(m_o - m_new);
+        float* st = sm_state + warp * kPartial;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) st[4 + 8 * hl + e] = o[e];
+        for (int e = 0; e < 8; ++e) {
+          const float oo = __shfl_xor_sync(0xffffffffu, o[e], 16);
+          if (hw % 2 == 0) st[4 + 8 * hl + e] = o[e] * a + oo * a_o;
+        }
+        if (lane == 0) {
+          st[0] = m_new;
+          st[1] = l_run * a + l_o * a_o;
+        }
       }
       worker_sync();
       if (tid < kDim) {
         float M = -INFINITY;
-        for (int k = 0; k < 2 * kWorkerWarps; ++k) M = fmaxf(M, sm_state[k * kPartial]);
+        for (int k = 0; k < kWorkerWarps; ++k) M = fmaxf(M, sm_state[k * kPartial]);
         float L = 0.0f, O = 0.0f;
         if (M != -INFINITY) {
-          for (int k = 0; k < 2 * kWorkerWarps; ++k) {
+          for (int k = 0; k < kWorkerWarps; ++k) {
             const float* sk = sm_state + k * kPartial;
             const float wgt = exp2f(sk[0] - M);  // 0 for a half-warp without rows
             L += sk[1] * wgt;

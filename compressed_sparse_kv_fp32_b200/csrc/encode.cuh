@@ -24,60 +24,116 @@ __device__ __forceinline__ uint32_t code_of(float y, float t0, float t2) {
   return 3u - (uint32_t)(y < t0) - (uint32_t)(y < 0.0f) - (uint32_t)(y < t2);
 }
 
-// ---------------------------------------------------------------- one vector per thread
-// v: the 128 elements in registers (constant indices only).
-template <int H>
-__device__ __forceinline__ void fwht_stage(float (&v)[kDim]) {
+// ---------------------------------------------------------------- one vector per thread, packed pairs
+// Packed fp32 pairs (sm_100): every element of the pair is rounded exactly as the
+// scalar operation would round it, so a pair instruction is two scalar operations
+// for one issue slot.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+
+// P[i] holds the elements (2i, 2i + 1) of one vector.  Stage h = 1 pairs the two
+// elements of one register and is done in scalar form as the bf16 words are
+// unpacked (rotate_pairs_first); stages h = 2 .. 64 pair register i with register
+// i + h/2 (bit h/2 of i clear), both of whose elements are butterfly partners.
+template <int HP>
+__device__ __forceinline__ void fwht_pair_stage(uint64_t (&P)[kDim / 2]) {
 #pragma unroll
-  for (int i = 0; i < kDim; i += 2 * H) {
+  for (int i = 0; i < kDim / 2; i += 2 * HP) {
 #pragma unroll
-    for (int j = i; j < i + H; ++j) {
-      const float a = v[j], b = v[j + H];
-      v[j] = __fadd_rn(a, b);
-      v[j + H] = __fsub_rn(a, b);
+    for (int j = i; j < i + HP; ++j) {
+      const uint64_t a = P[j], b = P[j + HP];
+      P[j] = f2_add(a, b);
+      P[j + HP] = f2_sub(a, b);
     }
   }
 }
 
-__device__ __forceinline__ void fwht128_thread(float (&v)[kDim]) {
-  fwht_stage<1>(v);
-  fwht_stage<2>(v);
-  fwht_stage<4>(v);
-  fwht_stage<8>(v);
-  fwht_stage<16>(v);
-  fwht_stage<32>(v);
-  fwht_stage<64>(v);
-  const float c = hadamard_norm();
-#pragma unroll
-  for (int j = 0; j < kDim; ++j) v[j] = __fmul_rn(v[j], c);
+// Stage h = 1 of the elements held in one packed bf16 word (elements 2i, 2i + 1).
+__device__ __forceinline__ uint64_t rotate_pair_first(uint32_t w) {
+  const float a = bf16_lo(w), b = bf16_hi(w);
+  return f2_pack(__fadd_rn(a, b), __fsub_rn(a, b));
 }
 
-// Rotated values -> 8 little-endian words of packed codes.
-// With z = y + 0 (turns -0 into +0, leaves every other value unchanged) and
-// h = m/2, the three comparisons are sign bits of exact sums: [y < -h] is the
-// sign of z + h, [y < 0] the sign of z, [y < h] the sign of z - h (a nonzero
-// exact sum of two floats never rounds to zero, and x - x = +0).  The code is
-// 3 minus their sum, so its high bit is NOT sign(z) and its low bit is
+// Stages h = 2 .. 64, then z = RN(y * C) for every element.  The normalisation is
+// one fused multiply-add with +0: its product is exact before the single rounding,
+// so z equals RN(y * C) bit for bit, except that a -0 result becomes +0 (which the
+// bucketing wants anyway; -0 and +0 compare equal).
+__device__ __forceinline__ void rotate_pairs_rest(uint64_t (&P)[kDim / 2]) {
+  fwht_pair_stage<1>(P);
+  fwht_pair_stage<2>(P);
+  fwht_pair_stage<4>(P);
+  fwht_pair_stage<8>(P);
+  fwht_pair_stage<16>(P);
+  fwht_pair_stage<32>(P);
+  const float c = hadamard_norm();
+  const uint64_t cc = f2_pack(c, c), zero = f2_pack(0.0f, 0.0f);
+#pragma unroll
+  for (int i = 0; i < kDim / 2; ++i) P[i] = f2_fma(P[i], cc, zero);
+}
+
+// Rotated values (pairs, -0 already +0) -> 8 little-endian words of packed codes.
+// With h = m/2 the three comparisons are sign bits of exact sums: [z < -h] is the
+// sign of z + h, [z < 0] the sign of z, [z < h] the sign of z - h (a nonzero exact
+// sum of two floats never rounds to zero, and x - x = +0).  The code is 3 minus
+// their sum, so its high bit is NOT sign(z) and its low bit is
 // NOT (sign(z + h) ^ sign(z) ^ sign(z - h)).  The bits are appended most
 // significant first with funnel shifts, inverted and byte-reversed at the end.
-__device__ __forceinline__ void bucket_pack_thread(const float (&y)[kDim], uint32_t (&w)[kCodeWords]) {
-  float m = 0.0f;
+__device__ __forceinline__ void bucket_pack_pairs(const uint64_t (&P)[kDim / 2], uint32_t (&w)[kCodeWords]) {
+  float mm[8];  // eight independent running maxima (short dependency chains)
 #pragma unroll
-  for (int i = 0; i < kDim; ++i) m = fmaxf(m, fabsf(y[i]));
+  for (int j = 0; j < 8; ++j) mm[j] = 0.0f;
+#pragma unroll
+  for (int i = 0; i < kDim / 2; ++i) {
+    float a, b;
+    f2_unpack(P[i], a, b);
+    mm[i & 7] = fmaxf(mm[i & 7], fmaxf(fabsf(a), fabsf(b)));
+  }
+  const float m = fmaxf(fmaxf(fmaxf(mm[0], mm[1]), fmaxf(mm[2], mm[3])), fmaxf(fmaxf(mm[4], mm[5]), fmaxf(mm[6], mm[7])));
   const float h = 0.5f * m;
+  const uint64_t hh = f2_pack(h, h);
+  // word i holds the codes of elements 16 i .. 16 i + 15 (pairs 8 i .. 8 i + 7)
+  uint32_t acc[kCodeWords];
+#pragma unroll
+  for (int i = 0; i < kCodeWords; ++i) acc[i] = 0u;
 #pragma unroll
   for (int i = 0; i < kCodeWords; ++i) {
-    uint32_t acc = 0;
 #pragma unroll
-    for (int e = 0; e < 16; ++e) {
-      const float z = __fadd_rn(y[16 * i + e], 0.0f);
-      const uint32_t zb = __float_as_uint(z);
-      const uint32_t lo = __float_as_uint(__fadd_rn(z, h)) ^ zb ^ __float_as_uint(__fsub_rn(z, h));
-      acc = __funnelshift_l(zb, acc, 1);
-      acc = __funnelshift_l(lo, acc, 1);
+    for (int q = 0; q < 8; ++q) {
+      const uint64_t z = P[8 * i + q];
+      float z0, z1, p0, p1, m0, m1;
+      f2_unpack(z, z0, z1);
+      f2_unpack(f2_add(z, hh), p0, p1);
+      f2_unpack(f2_sub(z, hh), m0, m1);
+      const uint32_t zb0 = __float_as_uint(z0), zb1 = __float_as_uint(z1);
+      acc[i] = __funnelshift_l(zb0, acc[i], 1);
+      acc[i] = __funnelshift_l(__float_as_uint(p0) ^ zb0 ^ __float_as_uint(m0), acc[i], 1);
+      acc[i] = __funnelshift_l(zb1, acc[i], 1);
+      acc[i] = __funnelshift_l(__float_as_uint(p1) ^ zb1 ^ __float_as_uint(m1), acc[i], 1);
     }
-    w[i] = __byte_perm(~acc, 0u, 0x0123);
   }
+#pragma unroll
+  for (int i = 0; i < kCodeWords; ++i) w[i] = __byte_perm(~acc[i], 0u, 0x0123);
 }
 
 // ---------------------------------------------------------------- one vector per warp

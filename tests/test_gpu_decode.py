@@ -65,7 +65,8 @@ TINY = [
     (1, 1, 1, 40000, [39999], 3000),
     # distances too many for shared memory: they go through the workspace
     (1, 8, 1, 200000, [200000], 512),
-    # many kept tokens per thread: per-thread phase-1 lists overflow and are rescanned
+    # budgets above the kept-list capacity (4096 tokens): the selection falls back to its
+    # two in-order scans, in windows of 4096 kept tokens
     (1, 32, 32, 40000, [40000], 8000),
     (1, 64, 32, 20000, [20000], 10000),
 ]

@@ -89,3 +89,33 @@ def test_append_negative_start_is_skipped(orc):
     want = np.zeros((1, 1, 8, 32), np.uint8)
     want[0, 0, :2] = orc.encode(x[0, 0, :2])
     assert np.array_equal(got, want)
+
+
+# ---- the prefill kernel (more than 8192 vectors per call): tiles of 32 rows per warp
+def test_prefill_special_vectors_tiled(orc):
+    x = special_vectors()
+    r = np.random.default_rng(11)
+    filler = synth.bf16_round(r.standard_normal((9000 - x.shape[0], 128)).astype(np.float32) * 3)
+    K = np.concatenate([x, filler])[None, None]                  # [1, 1, 9000, 128]
+    assert np.array_equal(gpu_encode(K)[0, 0], orc.encode(K[0, 0]))
+
+
+@pytest.mark.parametrize("n,count,start", [(1000, 1000, [0, 0, 0]),
+                                           (1000, 700, [0, 250, 900]),
+                                           (777, 777, [5, -40, 700]),
+                                           (2049, 1999, [1, 31, 33])])
+def test_prefill_ragged_windows(orc, n, count, start):
+    # 3 sequences x 5 kv heads, windows [start_b, start_b + count) clipped to [0, n);
+    # counts that are not multiples of 32 leave partial tiles at every head's end
+    r = np.random.default_rng(n + count)
+    B, Hkv = 3, 5
+    x = synth.bf16_round(r.standard_normal((B, Hkv, n, 128)).astype(np.float32) * 4)
+    codes = torch.full((B, Hkv, n, 32), 0xA5, dtype=torch.uint8, device="cuda")
+    got = gpu_encode(x, np.array(start, np.int32), count, codes)
+    want = np.full((B, Hkv, n, 32), 0xA5, dtype=np.uint8)
+    full = orc.encode(x)
+    for b in range(B):
+        lo, hi = max(0, start[b]), min(n, start[b] + count)
+        if hi > lo:
+            want[b, :, lo:hi] = full[b, :, lo:hi]
+    assert np.array_equal(got, want)
