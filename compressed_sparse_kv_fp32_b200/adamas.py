@@ -30,8 +30,29 @@ _lib = None
 SYMBOLS = (
     "adamas_status_string", "adamas_version", "adamas_last_error_string", "adamas_workspace_bytes", "adamas_workspace_init",
     "adamas_encode_keys", "adamas_decode_step", "adamas_score", "adamas_get_device_error",
-    "adamas_decode_step_static", "adamas_decode_step_append",
+    "adamas_decode_step_static", "adamas_decode_step_append", "adamas_decode_step_ex",
 )
+
+SELECT_PER_HEAD = 0
+SELECT_GROUP_SHARED = 1
+DEVERR_INTERNAL = 0x4
+DEVERR_TABLE = 0x8
+
+
+class DecodeArgs(ctypes.Structure):
+    """Mirror of adamas_decode_args (include/adamas.h), field for field."""
+
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("codes", ctypes.c_void_p), ("K", ctypes.c_void_p), ("V", ctypes.c_void_p),
+        ("seq_lens", ctypes.c_void_p),
+        ("B", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int), ("Nmax", ctypes.c_int64),
+        ("d", ctypes.c_int), ("budget", ctypes.c_int),
+        ("out", ctypes.c_void_p), ("idx", ctypes.c_void_p), ("workspace", ctypes.c_void_p),
+        ("workspace_bytes", ctypes.c_size_t),
+        ("append_pos", ctypes.c_void_p), ("k_new", ctypes.c_void_p), ("v_new", ctypes.c_void_p),
+        ("block_table", ctypes.c_void_p), ("n_pages", ctypes.c_int64), ("page_size", ctypes.c_int),
+        ("max_pages", ctypes.c_int), ("n_sink", ctypes.c_int), ("n_recent", ctypes.c_int), ("policy", ctypes.c_int),
+    ]
 
 
 class AdamasError(RuntimeError):
@@ -73,6 +94,8 @@ def load(path: str = LIBRARY) -> ctypes.CDLL:
         l.adamas_decode_step_static.restype = I
         l.adamas_decode_step_append.argtypes = [P, P, P, P, P, P, I, I, I, I64, I, I, P, P, P, SZ, P]
         l.adamas_decode_step_append.restype = I
+        l.adamas_decode_step_ex.argtypes = [ctypes.POINTER(DecodeArgs), P]
+        l.adamas_decode_step_ex.restype = I
         _lib = l
         return l
 
@@ -221,3 +244,65 @@ def score(q: torch.Tensor, codes: torch.Tensor, seq_lens: torch.Tensor, Hkv: Opt
     _check(load().adamas_score(q.data_ptr(), codes.data_ptr(), seq_lens.data_ptr(), B, Hq, Hkv, Nmax, d,
                                dist.data_ptr(), _stream(stream)), "adamas_score")
     return dist
+
+
+def decode(q: torch.Tensor, codes: torch.Tensor, K: torch.Tensor, V: torch.Tensor, seq_lens: torch.Tensor,
+           budget: int, workspace: Workspace, *, append_pos: Optional[torch.Tensor] = None,
+           k_new: Optional[torch.Tensor] = None, v_new: Optional[torch.Tensor] = None,
+           block_table: Optional[torch.Tensor] = None, n_sink: int = 0, n_recent: int = 0,
+           policy: int = SELECT_PER_HEAD, out: Optional[torch.Tensor] = None, idx: Optional[torch.Tensor] = None,
+           stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """adamas_decode_step_ex: the decode step with every option.
+
+    Contiguous cache: codes [B,Hkv,Nmax,32], K/V [B,Hkv,Nmax,128].  Paged cache
+    (block_table int32 [B, max_pages]): codes [n_pages,Hkv,P,32], K/V
+    [n_pages,Hkv,P,128] with P the page size.  append_pos int32 [B] encodes the key
+    at that position first; k_new/v_new bf16 [B,Hkv,128] are also written into the
+    cache there by the launch.  n_sink/n_recent force the first/last tokens of each
+    sequence into the kept set.  policy SELECT_GROUP_SHARED keeps one budget per kv
+    head (idx [B,Hkv,budget]).  Returns (out [B,Hq,128] fp32, idx)."""
+    _need(q, "q", torch.bfloat16)
+    if q.dim() != 3:
+        raise ValueError("q must be [B, Hq, 128]")
+    B, Hq, d = q.shape
+    _need(K, "K", torch.bfloat16)
+    if K.dim() != 4:
+        raise ValueError("K must be 4-dimensional")
+    paged = block_table is not None
+    if paged:
+        n_pages, Hkv, page_size, _ = K.shape
+        _need(block_table, "block_table", torch.int32)
+        if block_table.dim() != 2 or block_table.shape[0] != B:
+            raise ValueError("block_table must be [B, max_pages]")
+        max_pages = block_table.shape[1]
+        Nmax = max_pages * page_size
+        _need(K, "K", torch.bfloat16, (n_pages, Hkv, page_size, d))
+        _need(V, "V", torch.bfloat16, (n_pages, Hkv, page_size, d))
+        _need(codes, "codes", torch.uint8, (n_pages, Hkv, page_size, d // 4))
+    else:
+        _, Hkv, Nmax, _ = K.shape
+        n_pages = page_size = max_pages = 0
+        _need(K, "K", torch.bfloat16, (B, Hkv, Nmax, d))
+        _need(V, "V", torch.bfloat16, (B, Hkv, Nmax, d))
+        _need(codes, "codes", torch.uint8, (B, Hkv, Nmax, d // 4))
+    _need(seq_lens, "seq_lens", torch.int32, (B,))
+    rows = Hkv if policy == SELECT_GROUP_SHARED else Hq
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)
+    if idx is None:
+        idx = torch.empty((B, rows, budget), dtype=torch.int32, device=q.device)
+    _need(out, "out", torch.float32, (B, Hq, d))
+    _need(idx, "idx", torch.int32, (B, rows, budget))
+    if append_pos is not None:
+        _need(append_pos, "append_pos", torch.int32, (B,))
+    if (k_new is None) != (v_new is None):
+        raise ValueError("k_new and v_new go together")
+    if k_new is not None:
+        _need(k_new, "k_new", torch.bfloat16, (B, Hkv, d))
+        _need(v_new, "v_new", torch.bfloat16, (B, Hkv, d))
+    a = DecodeArgs(q.data_ptr(), codes.data_ptr(), K.data_ptr(), V.data_ptr(), seq_lens.data_ptr(),
+                   B, Hq, Hkv, Nmax, d, budget, out.data_ptr(), idx.data_ptr() if budget > 0 else None,
+                   workspace.buffer.data_ptr(), workspace.nbytes, _ptr(append_pos), _ptr(k_new), _ptr(v_new),
+                   _ptr(block_table), n_pages, page_size, max_pages, n_sink, n_recent, policy)
+    _check(load().adamas_decode_step_ex(ctypes.byref(a), _stream(stream)), "adamas_decode_step_ex")
+    return out, idx

@@ -12,7 +12,7 @@
 
 #include "../../include/adamas.h"
 #include "common.cuh"
-#include "decode.cuh"
+#include "decode_ext.cuh"
 #include "encode.cuh"
 #include "score.cuh"
 
@@ -210,10 +210,12 @@ struct OccEntry {
   int clusters;  // cudaOccupancyMaxActiveClusters
 };
 
+struct Plan;
+
 struct DeviceInfo {
   int sms = 0;
   size_t smem_optin = 0;
-  bool attrs_set[2][kMaxGroup + 1] = {};
+  bool attrs_set[3][2][kMaxGroup + 1] = {};  // [mode][smem_d][G]
   OccEntry occ[kOccCache] = {};
   int n_occ = 0;
   int enc_blocks_per_sm = 0;  // resident prefill-encoder blocks per SM (0: not yet set up)
@@ -254,13 +256,14 @@ static int device_info(DeviceInfo** out, int* dev_out = nullptr) {
 
 // One-time attributes of a decode kernel instance: the opt-in dynamic shared
 // memory and clusters of more than 8 blocks.
-static int kernel_attrs(DeviceInfo& dev, const void* fn, int G, bool smem_d) {
+static int kernel_attrs(DeviceInfo& dev, const void* fn, int G, bool smem_d, int mode) {
   std::lock_guard<std::mutex> lock(g_mutex);
-  if (dev.attrs_set[smem_d ? 1 : 0][G]) return ADAMAS_OK;
+  bool& done = dev.attrs_set[mode][smem_d ? 1 : 0][G];
+  if (done) return ADAMAS_OK;
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dev.smem_optin);
   if (e == cudaSuccess) e = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   if (e != cudaSuccess) return cuda_fail(e);
-  dev.attrs_set[smem_d ? 1 : 0][G] = true;
+  done = true;
   return ADAMAS_OK;
 }
 
@@ -312,22 +315,41 @@ static int active_clusters(DeviceInfo& dev, const void* fn, int cluster, size_t 
   return ADAMAS_OK;
 }
 
-template <int G, bool SMEM_D>
-static const void* decode_fn() {
-  return reinterpret_cast<const void*>(&decode_step_kernel<G, SMEM_D>);
+// Decode kernel instances live in one translation unit per group size.
+#define ADAMAS_DECL_G(N)                                                                            \
+  const void* decode_fn_g##N(bool smem_d, int mode);                                             \
+  cudaError_t decode_launch_g##N(const cudaLaunchConfig_t* cfg, const DecodeParams& prm, bool smem_d, \
+                                 int mode);
+ADAMAS_DECL_G(1) ADAMAS_DECL_G(2) ADAMAS_DECL_G(3) ADAMAS_DECL_G(4)
+ADAMAS_DECL_G(5) ADAMAS_DECL_G(6) ADAMAS_DECL_G(7) ADAMAS_DECL_G(8)
+#undef ADAMAS_DECL_G
+
+static const void* decode_fn_for(int G, bool smem_d, int mode) {
+  switch (G) {
+    case 1: return decode_fn_g1(smem_d, mode);
+    case 2: return decode_fn_g2(smem_d, mode);
+    case 3: return decode_fn_g3(smem_d, mode);
+    case 4: return decode_fn_g4(smem_d, mode);
+    case 5: return decode_fn_g5(smem_d, mode);
+    case 6: return decode_fn_g6(smem_d, mode);
+    case 7: return decode_fn_g7(smem_d, mode);
+    case 8: return decode_fn_g8(smem_d, mode);
+    default: return nullptr;
+  }
 }
 
-static const void* decode_fn_for(int G, bool smem_d) {
+static cudaError_t decode_launch_for(int G, const cudaLaunchConfig_t* cfg, const DecodeParams& prm, bool smem_d,
+                                     int mode) {
   switch (G) {
-    case 1: return smem_d ? decode_fn<1, true>() : decode_fn<1, false>();
-    case 2: return smem_d ? decode_fn<2, true>() : decode_fn<2, false>();
-    case 3: return smem_d ? decode_fn<3, true>() : decode_fn<3, false>();
-    case 4: return smem_d ? decode_fn<4, true>() : decode_fn<4, false>();
-    case 5: return smem_d ? decode_fn<5, true>() : decode_fn<5, false>();
-    case 6: return smem_d ? decode_fn<6, true>() : decode_fn<6, false>();
-    case 7: return smem_d ? decode_fn<7, true>() : decode_fn<7, false>();
-    case 8: return smem_d ? decode_fn<8, true>() : decode_fn<8, false>();
-    default: return nullptr;
+    case 1: return decode_launch_g1(cfg, prm, smem_d, mode);
+    case 2: return decode_launch_g2(cfg, prm, smem_d, mode);
+    case 3: return decode_launch_g3(cfg, prm, smem_d, mode);
+    case 4: return decode_launch_g4(cfg, prm, smem_d, mode);
+    case 5: return decode_launch_g5(cfg, prm, smem_d, mode);
+    case 6: return decode_launch_g6(cfg, prm, smem_d, mode);
+    case 7: return decode_launch_g7(cfg, prm, smem_d, mode);
+    case 8: return decode_launch_g8(cfg, prm, smem_d, mode);
+    default: return cudaErrorInvalidValue;
   }
 }
 
@@ -381,7 +403,7 @@ static bool layout_for(int G, int64_t Nmax, int cluster, size_t optin, Plan* P) 
 // Cluster size: the largest that keeps every cluster resident at once (one
 // wave), at most one block per SM in total, and at least kMinTokensPerBlock
 // tokens per block; 1 when even single blocks need several waves.
-static int make_plan(int B, int Hq, int Hkv, int64_t Nmax, DeviceInfo& dev, Plan* P) {
+static int make_plan_uncached(int B, int Hq, int Hkv, int64_t Nmax, int mode, DeviceInfo& dev, Plan* P) {
   const int G = Hq / Hkv;
   const int heads = B * Hkv;
   P->G = G;
@@ -394,8 +416,8 @@ static int make_plan(int B, int Hq, int Hkv, int64_t Nmax, DeviceInfo& dev, Plan
   for (int c = want; c >= 1 && !found; --c) {
     Plan t = *P;
     if (!layout_for(G, Nmax, c, dev.smem_optin, &t)) continue;
-    const void* fn = decode_fn_for(G, t.smem_d);
-    int rc = kernel_attrs(dev, fn, G, t.smem_d);
+    const void* fn = decode_fn_for(G, t.smem_d, mode);
+    int rc = kernel_attrs(dev, fn, G, t.smem_d, mode);
     if (rc != ADAMAS_OK) return rc;
     int n = 0;
     if ((rc = active_clusters(dev, fn, c, t.smem, &n)) != ADAMAS_OK) return rc;
@@ -414,10 +436,45 @@ static int make_plan(int B, int Hq, int Hkv, int64_t Nmax, DeviceInfo& dev, Plan
   return ADAMAS_OK;
 }
 
+// Plans of the shapes seen so far, per device (a decode loop calls with the same
+// shape every step: after the first call, planning is one table lookup).
+struct PlanKey {
+  int B, Hq, Hkv;
+  int64_t Nmax;
+  int mode;
+};
+constexpr int kPlanCache = 32;
+struct PlanCache {
+  PlanKey key[kPlanCache];
+  Plan plan[kPlanCache];
+  int n = 0, next = 0;
+};
+static PlanCache g_plans[kMaxDevices];
+
+static int make_plan(int B, int Hq, int Hkv, int64_t Nmax, int mode, DeviceInfo& dev, int devno, Plan* P) {
+  PlanCache& pc = g_plans[devno];
+  {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    for (int i = 0; i < pc.n; ++i) {
+      const PlanKey& k = pc.key[i];
+      if (k.B == B && k.Hq == Hq && k.Hkv == Hkv && k.Nmax == Nmax && k.mode == mode) {
+        *P = pc.plan[i];
+        return ADAMAS_OK;
+      }
+    }
+  }
+  const int rc = make_plan_uncached(B, Hq, Hkv, Nmax, mode, dev, P);
+  if (rc != ADAMAS_OK) return rc;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  const int slot = pc.n < kPlanCache ? pc.n++ : (pc.next++ % kPlanCache);
+  pc.key[slot] = PlanKey{B, Hq, Hkv, Nmax, mode};
+  pc.plan[slot] = *P;
+  return ADAMAS_OK;
+}
+
 static bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
 
-template <int G>
-static int launch_decode(const DecodeParams& prm, const Plan& P, cudaStream_t stream) {
+static int launch_decode(const DecodeParams& prm, const Plan& P, int mode, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)P.grid);
   cfg.blockDim = dim3(kThreads);
@@ -434,70 +491,96 @@ static int launch_decode(const DecodeParams& prm, const Plan& P, cudaStream_t st
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  const cudaError_t e = P.smem_d ? cudaLaunchKernelEx(&cfg, decode_step_kernel<G, true>, prm)
-                                 : cudaLaunchKernelEx(&cfg, decode_step_kernel<G, false>, prm);
+  cudaError_t e = decode_launch_for(P.G, &cfg, prm, P.smem_d, mode);
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
   return ADAMAS_OK;
 }
 
-// Argument checks shared by both decode entry points (before anything is enqueued).
-static int check_decode_args(const void* q, const uint8_t* codes, const void* K, const void* V,
-                             const int32_t* seq_lens, int B, int Hq, int Hkv, int64_t Nmax, int d, int budget,
-                             const float* out, const int32_t* idx) {
-  int rc = check_shape(B, Hq, Hkv, Nmax, d, budget);
+// Argument checks of a decode call (before anything is enqueued).  Fills *Nmax_out
+// with the tokens a sequence can hold (paged: max_pages * page_size).
+static int check_decode_args(const adamas_decode_args& a, int64_t* Nmax_out) {
+  const bool paged = a.block_table != nullptr;
+  int64_t Nmax = a.Nmax;
+  if (paged) {
+    if (a.page_size < 1 || a.max_pages < 1 || a.n_pages < 1) return ADAMAS_ERR_INVALID_ARG;
+    Nmax = (int64_t)a.max_pages * a.page_size;
+    if (Nmax > INT32_MAX || a.n_pages * a.Hkv * (int64_t)a.page_size > INT32_MAX) return ADAMAS_ERR_UNSUPPORTED;
+    if (!aligned(a.block_table, 4)) return ADAMAS_ERR_INVALID_ARG;
+  }
+  *Nmax_out = Nmax;
+  int rc = check_shape(a.B, a.Hq, a.Hkv, Nmax, a.d, a.budget);
   if (rc != ADAMAS_OK) return rc;
-  if (B == 0) return ADAMAS_OK;
-  if (!q || !seq_lens || !out || (budget > 0 && !idx)) return ADAMAS_ERR_INVALID_ARG;
-  if (Nmax > 0 && (!codes || !K || !V)) return ADAMAS_ERR_INVALID_ARG;
-  if (!aligned(q, 16) || !aligned(codes, 32) || !aligned(K, 16) || !aligned(V, 16) || !aligned(out, 16) ||
-      !aligned(idx, 4) || !aligned(seq_lens, 4))
+  if (a.policy != ADAMAS_SELECT_PER_HEAD && a.policy != ADAMAS_SELECT_GROUP_SHARED) return ADAMAS_ERR_INVALID_ARG;
+  if (a.policy == ADAMAS_SELECT_GROUP_SHARED && a.budget > kKeptCap) return ADAMAS_ERR_UNSUPPORTED;
+  if (a.n_sink < 0 || a.n_recent < 0) return ADAMAS_ERR_INVALID_ARG;
+  if (a.B == 0) return ADAMAS_OK;
+  if (!a.q || !a.seq_lens || !a.out || (a.budget > 0 && !a.idx)) return ADAMAS_ERR_INVALID_ARG;
+  if (Nmax > 0 && (!a.codes || !a.K || !a.V)) return ADAMAS_ERR_INVALID_ARG;
+  if (!aligned(a.q, 16) || !aligned(a.codes, 32) || !aligned(a.K, 16) || !aligned(a.V, 16) || !aligned(a.out, 16) ||
+      !aligned(a.idx, 4) || !aligned(a.seq_lens, 4))
     return ADAMAS_ERR_INVALID_ARG;
+  if ((a.k_new == nullptr) != (a.v_new == nullptr)) return ADAMAS_ERR_INVALID_ARG;
+  if (a.k_new && (!a.append_pos || !aligned(a.k_new, 16) || !aligned(a.v_new, 16))) return ADAMAS_ERR_INVALID_ARG;
+  if (a.append_pos && !aligned(a.append_pos, 4)) return ADAMAS_ERR_INVALID_ARG;
   return ADAMAS_OK;
 }
 
-// Enqueue the decode kernel with its scratch at `ws` (laid out by `P`); with
-// append_pos, the keys at those positions are encoded into codes first.
-static int enqueue_decode(const void* q, const uint8_t* codes, const void* K, const void* V,
-                          const int32_t* seq_lens, int B, int Hq, int Hkv, int64_t Nmax, int budget, float* out,
-                          int32_t* idx, unsigned char* ws, const Plan& P, cudaStream_t st,
-                          const int32_t* append_pos = nullptr) {
-  DecodeParams prm;
-  prm.q = static_cast<const uint16_t*>(q);
-  prm.codes = codes;
-  prm.K = static_cast<const uint16_t*>(K);
-  prm.V = static_cast<const uint16_t*>(V);
-  prm.seq_lens = seq_lens;
-  prm.out = out;
-  prm.idx = idx;
+// The kernel instance a call needs: group-shared, general (any option), or plain.
+static int decode_mode(const adamas_decode_args& a) {
+  if (a.policy == ADAMAS_SELECT_GROUP_SHARED) return kModeShared;
+  if (a.block_table || a.k_new || a.n_sink > 0 || a.n_recent > 0) return kModeGeneral;
+  return kModePlain;
+}
+
+// Enqueue the decode kernel with its scratch at `ws` (laid out by `P`).
+static int enqueue_decode(const adamas_decode_args& a, int64_t Nmax, unsigned char* ws, const Plan& P,
+                          cudaStream_t st) {
+  DecodeParams prm = {};
+  prm.q = static_cast<const uint16_t*>(a.q);
+  prm.codes = a.codes;
+  prm.K = static_cast<const uint16_t*>(a.K);
+  prm.V = static_cast<const uint16_t*>(a.V);
+  prm.seq_lens = a.seq_lens;
+  prm.out = a.out;
+  prm.idx = a.idx;
   prm.err = reinterpret_cast<uint32_t*>(ws + P.ctrl) + 2;
   prm.dglobal = P.smem_d ? nullptr : reinterpret_cast<uint16_t*>(ws + P.dspill);
-  prm.codes_w = append_pos ? const_cast<uint8_t*>(codes) : nullptr;
-  prm.append_pos = append_pos;
-  prm.B = B;
-  prm.Hq = Hq;
-  prm.Hkv = Hkv;
+  prm.codes_w = a.append_pos ? a.codes : nullptr;
+  prm.append_pos = a.append_pos;
+  prm.k_new = static_cast<const uint16_t*>(a.k_new);
+  prm.v_new = static_cast<const uint16_t*>(a.v_new);
+  prm.K_w = a.k_new ? static_cast<uint16_t*>(a.K) : nullptr;
+  prm.V_w = a.k_new ? static_cast<uint16_t*>(a.V) : nullptr;
+  prm.table = a.block_table;
+  prm.n_pages = a.block_table ? a.n_pages : 0;
+  prm.page_size = a.block_table ? a.page_size : 1;
+  prm.max_pages = a.block_table ? a.max_pages : 0;
+  prm.n_sink = a.n_sink;
+  prm.n_recent = a.n_recent;
+  prm.B = a.B;
+  prm.Hq = a.Hq;
+  prm.Hkv = a.Hkv;
   prm.Nmax = Nmax;
-  prm.budget = budget;
+  prm.budget = a.budget;
   prm.cluster = P.cluster;
   prm.nstages = P.nstages;
   prm.dstride = P.dstride;
-  int rc;
-  switch (P.G) {
-    case 1: rc = launch_decode<1>(prm, P, st); break;
-    case 2: rc = launch_decode<2>(prm, P, st); break;
-    case 3: rc = launch_decode<3>(prm, P, st); break;
-    case 4: rc = launch_decode<4>(prm, P, st); break;
-    case 5: rc = launch_decode<5>(prm, P, st); break;
-    case 6: rc = launch_decode<6>(prm, P, st); break;
-    case 7: rc = launch_decode<7>(prm, P, st); break;
-    case 8: rc = launch_decode<8>(prm, P, st); break;
-    default: rc = ADAMAS_ERR_UNSUPPORTED;
-  }
-  if (rc == ADAMAS_OK) {
-    const cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) rc = cuda_fail(e);
-  }
-  return rc;
+  return launch_decode(prm, P, decode_mode(a), st);
+}
+
+// A decode call on a caller workspace: checks, plan, launch.
+static int decode_with_workspace(const adamas_decode_args& a, cudaStream_t st) {
+  int64_t Nmax = 0;
+  int rc = check_decode_args(a, &Nmax);
+  if (rc != ADAMAS_OK || a.B == 0) return rc;
+  DeviceInfo* dev = nullptr;
+  int devno = 0;
+  if ((rc = device_info(&dev, &devno)) != ADAMAS_OK) return rc;
+  Plan P;
+  if ((rc = make_plan(a.B, a.Hq, a.Hkv, Nmax, decode_mode(a), *dev, devno, &P)) != ADAMAS_OK) return rc;
+  if (!a.workspace || a.workspace_bytes < P.total || !aligned(a.workspace, 16)) return ADAMAS_ERR_WORKSPACE;
+  return enqueue_decode(a, Nmax, static_cast<unsigned char*>(a.workspace), P, st);
 }
 
 template <int G>
@@ -533,9 +616,10 @@ const char* adamas_last_error_string(void) {
 size_t adamas_workspace_bytes(int B, int Hq, int Hkv, int64_t Nmax, int d, int budget) {
   if (check_shape(B, Hq, Hkv, Nmax, d, budget) != ADAMAS_OK) return 0;
   DeviceInfo* dev = nullptr;
-  if (device_info(&dev) != ADAMAS_OK) return 0;
+  int devno = 0;
+  if (device_info(&dev, &devno) != ADAMAS_OK) return 0;
   Plan P;
-  if (make_plan(B, Hq, Hkv, Nmax, *dev, &P) != ADAMAS_OK) return 0;
+  if (make_plan(B, Hq, Hkv, Nmax, kModePlain, *dev, devno, &P) != ADAMAS_OK) return 0;
   return P.total;
 }
 
@@ -548,9 +632,10 @@ int adamas_workspace_init(void* workspace, size_t workspace_bytes, adamas_stream
 
 int adamas_encode_keys(const void* K, uint8_t* codes, const int32_t* pos_begin, int count, int B, int Hkv,
                        int64_t Nmax, int d, adamas_stream_t stream) {
-  const int rc = check_shape(B, Hkv, Hkv, Nmax, d, 0);
-  if (rc != ADAMAS_OK) return rc;
-  if (count < 0) return ADAMAS_ERR_INVALID_ARG;
+  // no batch limit here: the pages of a paged cache are encoded as B = n_pages sequences
+  if (B < 0 || Hkv <= 0 || Nmax < 0 || count < 0) return ADAMAS_ERR_INVALID_ARG;
+  if (d != kDim) return ADAMAS_ERR_UNSUPPORTED;
+  if (Nmax > INT32_MAX || (int64_t)B * Hkv > INT32_MAX) return ADAMAS_ERR_UNSUPPORTED;
   if (B == 0 || count == 0 || Nmax == 0) return ADAMAS_OK;
   if (!K || !codes || !aligned(K, 16) || !aligned(codes, 32)) return ADAMAS_ERR_INVALID_ARG;
   if (pos_begin && !aligned(pos_begin, 4)) return ADAMAS_ERR_INVALID_ARG;
@@ -579,36 +664,53 @@ int adamas_encode_keys(const void* K, uint8_t* codes, const int32_t* pos_begin, 
   return ADAMAS_OK;
 }
 
+// The plain calls below are adamas_decode_step_ex with the optional fields unset.
+static adamas_decode_args plain_args(const void* q, const uint8_t* codes, const void* K, const void* V,
+                                     const int32_t* seq_lens, int B, int Hq, int Hkv, int64_t Nmax, int d, int budget,
+                                     float* out, int32_t* idx, void* workspace, size_t workspace_bytes) {
+  adamas_decode_args a;
+  memset(&a, 0, sizeof a);
+  a.q = q;
+  a.codes = const_cast<uint8_t*>(codes);
+  a.K = const_cast<void*>(K);
+  a.V = const_cast<void*>(V);
+  a.seq_lens = seq_lens;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.Nmax = Nmax;
+  a.d = d;
+  a.budget = budget;
+  a.out = out;
+  a.idx = idx;
+  a.workspace = workspace;
+  a.workspace_bytes = workspace_bytes;
+  a.policy = ADAMAS_SELECT_PER_HEAD;
+  return a;
+}
+
 int adamas_decode_step(const void* q, const uint8_t* codes, const void* K, const void* V, const int32_t* seq_lens,
                        int B, int Hq, int Hkv, int64_t Nmax, int d, int budget, float* out, int32_t* idx,
                        void* workspace, size_t workspace_bytes, adamas_stream_t stream) {
-  int rc = check_decode_args(q, codes, K, V, seq_lens, B, Hq, Hkv, Nmax, d, budget, out, idx);
-  if (rc != ADAMAS_OK || B == 0) return rc;
-  DeviceInfo* dev = nullptr;
-  if ((rc = device_info(&dev)) != ADAMAS_OK) return rc;
-  Plan P;
-  if ((rc = make_plan(B, Hq, Hkv, Nmax, *dev, &P)) != ADAMAS_OK) return rc;
-  if (!workspace || workspace_bytes < P.total || !aligned(workspace, 16)) return ADAMAS_ERR_WORKSPACE;
-  return enqueue_decode(q, codes, K, V, seq_lens, B, Hq, Hkv, Nmax, budget, out, idx,
-                        static_cast<unsigned char*>(workspace), P, (cudaStream_t)stream);
+  const adamas_decode_args a =
+      plain_args(q, codes, K, V, seq_lens, B, Hq, Hkv, Nmax, d, budget, out, idx, workspace, workspace_bytes);
+  return decode_with_workspace(a, (cudaStream_t)stream);
 }
 
 int adamas_decode_step_append(const void* q, uint8_t* codes, const void* K, const void* V, const int32_t* seq_lens,
                               const int32_t* append_pos, int B, int Hq, int Hkv, int64_t Nmax, int d, int budget,
                               float* out, int32_t* idx, void* workspace, size_t workspace_bytes,
                               adamas_stream_t stream) {
-  int rc = check_decode_args(q, codes, K, V, seq_lens, B, Hq, Hkv, Nmax, d, budget, out, idx);
-  if (rc != ADAMAS_OK || B == 0) return rc;
-  if (!append_pos || !aligned(append_pos, 4)) return ADAMAS_ERR_INVALID_ARG;
-  if (Nmax == 0) return adamas_decode_step(q, codes, K, V, seq_lens, B, Hq, Hkv, Nmax, d, budget, out, idx, workspace,
-                                           workspace_bytes, stream);
-  DeviceInfo* dev = nullptr;
-  if ((rc = device_info(&dev)) != ADAMAS_OK) return rc;
-  Plan P;
-  if ((rc = make_plan(B, Hq, Hkv, Nmax, *dev, &P)) != ADAMAS_OK) return rc;
-  if (!workspace || workspace_bytes < P.total || !aligned(workspace, 16)) return ADAMAS_ERR_WORKSPACE;
-  return enqueue_decode(q, codes, K, V, seq_lens, B, Hq, Hkv, Nmax, budget, out, idx,
-                        static_cast<unsigned char*>(workspace), P, (cudaStream_t)stream, append_pos);
+  if (B > 0 && !append_pos) return ADAMAS_ERR_INVALID_ARG;
+  adamas_decode_args a =
+      plain_args(q, codes, K, V, seq_lens, B, Hq, Hkv, Nmax, d, budget, out, idx, workspace, workspace_bytes);
+  a.append_pos = append_pos;
+  return decode_with_workspace(a, (cudaStream_t)stream);
+}
+
+int adamas_decode_step_ex(const adamas_decode_args* args, adamas_stream_t stream) {
+  if (!args) return ADAMAS_ERR_INVALID_ARG;
+  return decode_with_workspace(*args, (cudaStream_t)stream);
 }
 
 int adamas_score(const void* q, const uint8_t* codes, const int32_t* seq_lens, int B, int Hq, int Hkv, int64_t Nmax,
@@ -696,12 +798,15 @@ static int static_scratch(void** out) {
 extern "C" int adamas_decode_step_static(const void* q, const uint8_t* codes, const void* K, const void* V,
                                          const int32_t* seq_lens, int B, int Hq, int Hkv, int64_t Nmax, int d,
                                          int budget, float* out, int32_t* idx, adamas_stream_t stream) {
-  int rc = check_decode_args(q, codes, K, V, seq_lens, B, Hq, Hkv, Nmax, d, budget, out, idx);
+  const adamas_decode_args a = plain_args(q, codes, K, V, seq_lens, B, Hq, Hkv, Nmax, d, budget, out, idx, nullptr, 0);
+  int64_t Nm = 0;
+  int rc = check_decode_args(a, &Nm);
   if (rc != ADAMAS_OK || B == 0) return rc;
   DeviceInfo* dev = nullptr;
-  if ((rc = device_info(&dev)) != ADAMAS_OK) return rc;
+  int devno = 0;
+  if ((rc = device_info(&dev, &devno)) != ADAMAS_OK) return rc;
   Plan P;
-  if ((rc = make_plan(B, Hq, Hkv, Nmax, *dev, &P)) != ADAMAS_OK) return rc;
+  if ((rc = make_plan(B, Hq, Hkv, Nm, kModePlain, *dev, devno, &P)) != ADAMAS_OK) return rc;
   if (P.total > kStaticScratchBytes) return ADAMAS_ERR_WORKSPACE;  // sizes beyond the fixed scratch
   void* scratch = nullptr;
   if ((rc = static_scratch(&scratch)) != ADAMAS_OK) return rc;
@@ -710,6 +815,5 @@ extern "C" int adamas_decode_step_static(const void* q, const uint8_t* codes, co
   cudaStream_t st = (cudaStream_t)stream;
   const cudaError_t e = cudaMemsetAsync(scratch, 0, P.dspill, st);
   if (e != cudaSuccess) return cuda_fail(e);
-  return enqueue_decode(q, codes, K, V, seq_lens, B, Hq, Hkv, Nmax, budget, out, idx,
-                        static_cast<unsigned char*>(scratch), P, st);
+  return enqueue_decode(a, Nm, static_cast<unsigned char*>(scratch), P, st);
 }

@@ -17,6 +17,7 @@ constexpr int kMaxBatch = 1024;
 constexpr uint32_t kErrSeqLen = 0x1u;
 constexpr uint32_t kErrTimeout = 0x2u;
 constexpr uint32_t kErrInternal = 0x4u;
+constexpr uint32_t kErrTable = 0x8u;
 
 // RN_fp32(1/sqrt(128)), bit pattern 0x3DB504F3: the rotation's normalisation.
 __device__ __forceinline__ float hadamard_norm() { return __uint_as_float(0x3DB504F3u); }

@@ -65,6 +65,13 @@ enum adamas_status {
 #define ADAMAS_DEVERR_SEQLEN 0x1u  /* a seq_lens entry was outside [0, Nmax]; it was clamped */
 #define ADAMAS_DEVERR_TIMEOUT 0x2u /* a bounded wait on a stage copy gave up; the step's outputs are invalid */
 #define ADAMAS_DEVERR_INTERNAL 0x4u /* a block's share exceeded its planned size; outputs are invalid */
+#define ADAMAS_DEVERR_TABLE 0x8u    /* a block-table entry was outside [0, n_pages); page 0 was read instead */
+
+/* Selection policies of adamas_decode_step_ex. */
+enum adamas_select_policy {
+    ADAMAS_SELECT_PER_HEAD = 0,    /* every query head keeps its own budget of tokens */
+    ADAMAS_SELECT_GROUP_SHARED = 1 /* one budget per kv head, ranked by the distance summed over its query heads */
+};
 
 /* Static description of a status code (never NULL). */
 const char *adamas_status_string(int status);
@@ -189,6 +196,78 @@ int adamas_score(const void *q, const uint8_t *codes, const int32_t *seq_lens, i
 int adamas_decode_step_static(const void *q, const uint8_t *codes, const void *K, const void *V,
                               const int32_t *seq_lens, int B, int Hq, int Hkv, int64_t Nmax, int d,
                               int budget, float *out, int32_t *idx, adamas_stream_t stream);
+
+/*
+ * Every option of the decode step in one call.  adamas_decode_step and
+ * adamas_decode_step_append are this call with the optional fields zero.
+ *
+ * Required fields (as in adamas_decode_step):
+ *   q, codes, K, V, seq_lens, B, Hq, Hkv, Nmax, d, budget, out, idx,
+ *   workspace, workspace_bytes
+ *
+ * Optional fields (zero / NULL: off):
+ *   append_pos   device int32 [B]: the key at append_pos[b] is encoded into codes
+ *                before the step scores it (adamas_decode_step_append; the ADAMAS
+ *                article's §3.1: the code cache grows by one row per token).
+ *   k_new, v_new device bf16 [B][Hkv][128], both or neither, only with append_pos:
+ *                the launch itself writes these rows into K and V at append_pos[b]
+ *                (and encodes k_new), so a decode loop needs no separate copy of the
+ *                new token's rows into the cache.  K and V are written.
+ *   block_table  device int32 [B][max_pages]: a paged cache.  Token t of sequence b
+ *                lives in physical page block_table[b][t / page_size] at slot
+ *                t % page_size; codes, K and V are then page arrays laid out
+ *                [n_pages][Hkv][page_size][32 or 128] (every kv head's rows of a page
+ *                contiguous), and Nmax is ignored (max_pages * page_size tokens per
+ *                sequence).  adamas_encode_keys encodes such a cache as B = n_pages
+ *                sequences of Nmax = page_size tokens.  An entry outside
+ *                [0, n_pages) sets ADAMAS_DEVERR_TABLE (the step then reads page 0).
+ *                Requires n_pages * Hkv * page_size <= 2^31 - 1.
+ *   page_size, max_pages, n_pages   the paged cache's geometry.
+ *   n_sink, n_recent  forced rows: the first n_sink and the last n_recent tokens of
+ *                every sequence rank ahead of every scored token (in index order), as
+ *                attention sinks and a recent window; the rest are ranked by (D, t).
+ *                When they outnumber k_eff the lowest indices win.
+ *   policy       ADAMAS_SELECT_PER_HEAD (default) or ADAMAS_SELECT_GROUP_SHARED: for
+ *                every (b, kv head) the distances of its G query heads are summed per
+ *                token, k_eff tokens of smallest (sum, t) are kept once, and every
+ *                query head of the group attends over them; idx is then
+ *                [B][Hkv][budget] and budget must be <= 4096 (ADAMAS_ERR_UNSUPPORTED
+ *                otherwise).  The K/V rows are read once per kv head instead of once
+ *                per query head.
+ * The grouped-head and forced-row rules are readings of the article's §2.3 and
+ * §5.2 (which state the scoring and the budget per head) and of its §3.2 and §6
+ * tuning advice (some tokens keep full attention); the paged layout follows the
+ * block-table caches that paged-attention serving uses.  Same errors and
+ * asynchrony as adamas_decode_step; the workspace size is adamas_workspace_bytes of
+ * (B, Hq, Hkv, Nmax, d, budget) with Nmax = max_pages * page_size when paged.
+ */
+typedef struct adamas_decode_args {
+    const void *q;
+    uint8_t *codes;
+    void *K;
+    void *V;
+    const int32_t *seq_lens;
+    int B, Hq, Hkv;
+    int64_t Nmax;
+    int d;
+    int budget;
+    float *out;
+    int32_t *idx;
+    void *workspace;
+    size_t workspace_bytes;
+    const int32_t *append_pos;
+    const void *k_new;
+    const void *v_new;
+    const int32_t *block_table;
+    int64_t n_pages;
+    int page_size;
+    int max_pages;
+    int n_sink;
+    int n_recent;
+    int policy;
+} adamas_decode_args;
+
+int adamas_decode_step_ex(const adamas_decode_args *args, adamas_stream_t stream);
 
 /*
  * Synchronise `stream`, then copy the workspace's device error word into

@@ -236,19 +236,29 @@ def decode_step_forced(q, K, V, codes, seq_lens, budget: int, n_sink: int, n_rec
 
 def decode_step_paged(q, K_pages, V_pages, code_pages, block_table, seq_lens, budget: int):
     """Per-head decode step over a paged cache: token t of sequence b lives in
-    physical page block_table[b, t // P] at offset t % P (P = page size, the
-    pages' second dimension).  K_pages/V_pages [n_pages, P, Hkv, 128] bf16 bits,
-    code_pages [n_pages, P, Hkv, 32], block_table int32 [B, max_pages].  The
-    tokens are read through the table into sequence order and the plain step
-    runs on them.  Returns (out float64 [B,Hq,128], idx int32 [B,Hq,budget])."""
+    physical page block_table[b, t // P] at slot t % P (P = page size).  Pages are
+    laid out with every kv head's rows of a page contiguous: K_pages/V_pages
+    [n_pages, Hkv, P, 128] bf16 bits, code_pages [n_pages, Hkv, P, 32], block_table
+    int32 [B, max_pages].  The tokens are read through the table into sequence
+    order and the plain step runs on them.  Returns (out float64 [B,Hq,128], idx
+    int32 [B,Hq,budget])."""
+    K, V, codes, lens = paged_to_contiguous(K_pages, V_pages, code_pages, block_table, seq_lens)
+    out, idx, _ = decode_step(q, K, V, codes, lens, budget)
+    return out, idx
+
+
+def paged_to_contiguous(K_pages, V_pages, code_pages, block_table, seq_lens):
+    """The contiguous cache [B, Hkv, max_pages * P, ...] that a paged cache describes
+    (positions past each sequence's length are zero).  Raises on a table entry
+    outside [0, n_pages) within a sequence."""
     K_pages = _c(K_pages, np.uint16)
     V_pages = _c(V_pages, np.uint16)
     code_pages = _c(code_pages, np.uint8)
     table = _c(block_table, np.int32)
     lens = _c(seq_lens, np.int32)
-    n_pages, P, Hkv, d = K_pages.shape
+    n_pages, Hkv, P, d = K_pages.shape
     B, max_pages = table.shape
-    if V_pages.shape != K_pages.shape or code_pages.shape != (n_pages, P, Hkv, 32) or lens.shape != (B,):
+    if V_pages.shape != K_pages.shape or code_pages.shape != (n_pages, Hkv, P, 32) or lens.shape != (B,):
         raise ValueError("oracle: inconsistent shapes")
     Nmax = max_pages * P
     K = np.zeros((B, Hkv, Nmax, d), dtype=np.uint16)
@@ -262,8 +272,58 @@ def decode_step_paged(q, K_pages, V_pages, code_pages, block_table, seq_lens, bu
             page = int(table[b, t // P])
             if not 0 <= page < n_pages:
                 raise ValueError("oracle: block table entry out of range")
-            K[b, :, t] = K_pages[page, t % P]
-            V[b, :, t] = V_pages[page, t % P]
-            codes[b, :, t] = code_pages[page, t % P]
-    out, idx, _ = decode_step(q, K, V, codes, lens, budget)
+            K[b, :, t] = K_pages[page, :, t % P]
+            V[b, :, t] = V_pages[page, :, t % P]
+            codes[b, :, t] = code_pages[page, :, t % P]
+    return K, V, codes, lens
+
+
+def decode_step_general(q, K, V, codes, seq_lens, budget: int, n_sink: int = 0, n_recent: int = 0,
+                        group_shared: bool = False):
+    """Decode step with forced rows and/or group-shared selection together (the
+    rules of decode_step_forced and decode_step_group_shared combined): per token
+    the ranking distance is -1 for a forced row, else its L1 distance (summed over
+    the group's query heads when group_shared); k_eff = min(budget, len) tokens of
+    smallest (distance, index) are kept, per query head or once per kv head.
+    Returns (out float64 [B,Hq,128], idx int32 [B,Hq or Hkv,budget])."""
+    q = _c(q, np.uint16)
+    K = _c(K, np.uint16)
+    V = _c(V, np.uint16)
+    codes = _c(codes, np.uint8)
+    lens = _c(seq_lens, np.int32)
+    B, Hq, d = q.shape
+    _, Hkv, Nmax, _ = K.shape
+    if Hq % Hkv or V.shape != K.shape or codes.shape != (B, Hkv, Nmax, 32) or lens.shape != (B,):
+        raise ValueError("oracle: inconsistent shapes")
+    if n_sink < 0 or n_recent < 0:
+        raise ValueError("oracle: negative forced-row counts")
+    G = Hq // Hkv
+    qcodes = encode(q.reshape(-1, d)).reshape(B, Hq, 32)
+    out = np.zeros((B, Hq, d), dtype=np.float64)
+    idx = np.full((B, Hkv if group_shared else Hq, budget), -1, dtype=np.int32)
+    for b in range(B):
+        n = int(lens[b])
+        if n < 0 or n > Nmax:
+            raise ValueError("oracle: sequence length outside [0, Nmax]")
+        keff = min(budget, n)
+        if keff == 0:
+            continue
+        t = np.arange(n)
+        forced = (t < n_sink) | (t >= n - n_recent)
+        for h in range(Hkv):
+            Ds = [distance(qcodes[b, h * G + g], codes[b, h, :n]).astype(np.int64) for g in range(G)]
+            if group_shared:
+                D = np.sum(Ds, axis=0)
+                D[forced] = -1
+                kept = select(D.astype(np.int32), keff)
+                idx[b, h, :keff] = kept
+                for g in range(G):
+                    out[b, h * G + g] = attend(q[b, h * G + g], K[b, h, :n], V[b, h, :n], kept)
+            else:
+                for g in range(G):
+                    D = Ds[g].copy()
+                    D[forced] = -1
+                    kept = select(D.astype(np.int32), keff)
+                    idx[b, h * G + g, :keff] = kept
+                    out[b, h * G + g] = attend(q[b, h * G + g], K[b, h, :n], V[b, h, :n], kept)
     return out, idx

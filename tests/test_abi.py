@@ -72,3 +72,37 @@ def test_host_side_argument_errors(lib):
     assert lib.adamas_decode_step(None, None, None, None, None, 0, 4, 4, 64, 128, 8, None, None,
                                   None, 0, None) == 0
     assert lib.adamas_encode_keys(None, None, None, 0, 1, 4, 64, 128, None) == 0
+
+
+def test_decode_args_layout_matches_the_header(tmp_path):
+    # the ctypes mirror of adamas_decode_args must agree with the C compiler's layout
+    fields = [f for f, _ in adamas.DecodeArgs._fields_]
+    prog = tmp_path / "layout.c"
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "adamas.h"', 'int main(void) {',
+             '  printf("%zu\\n", sizeof(adamas_decode_args));']
+    lines += [f'  printf("%zu\\n", offsetof(adamas_decode_args, {f}));' for f in fields]
+    lines += ['  return 0;', '}']
+    prog.write_text("\n".join(lines))
+    exe = tmp_path / "layout"
+    import subprocess
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), "-o", str(exe), str(prog)], check=True)
+    got = [int(x) for x in subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()]
+    assert got[0] == ctypes.sizeof(adamas.DecodeArgs)
+    assert got[1:] == [getattr(adamas.DecodeArgs, f).offset for f in fields]
+
+
+def test_decode_ex_rejects_bad_options_before_any_launch(lib):
+    fake = 1 << 20                                   # never dereferenced: the checks come first
+    base = dict(q=fake, codes=fake, K=fake, V=fake, seq_lens=fake, B=1, Hq=4, Hkv=1, Nmax=4096, d=128, budget=64,
+                out=fake, idx=fake, workspace=fake, workspace_bytes=1 << 20, policy=0)
+    def call(**kw):
+        a = adamas.DecodeArgs(**dict(base, **kw))
+        return lib.adamas_decode_step_ex(ctypes.byref(a), None)
+    assert call(policy=7) == -1                      # unknown policy
+    assert call(policy=1, budget=5000) == -2         # group-shared budget above 4096
+    assert call(n_sink=-1) == -1
+    assert call(k_new=fake) == -1                    # k_new without v_new
+    assert call(k_new=fake, v_new=fake) == -1        # rows without append positions
+    assert call(block_table=fake, page_size=0, max_pages=4, n_pages=8) == -1
+    assert call(block_table=fake + 2, page_size=16, max_pages=4, n_pages=8) == -1   # misaligned table
+    assert lib.adamas_decode_step_ex(None, None) == -1

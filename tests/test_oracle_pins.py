@@ -501,16 +501,16 @@ def test_paged_step_equals_the_contiguous_step(orc):
     rng = np.random.default_rng(5)
     n_pages = 3 * max_pages + 4
     perm = rng.permutation(n_pages)[:3 * max_pages].reshape(3, max_pages).astype(np.int32)
-    Kp = rng.integers(0, 2 ** 16, size=(n_pages, P, 2, 128), dtype=np.uint16)  # garbage where unused
-    Vp = rng.integers(0, 2 ** 16, size=(n_pages, P, 2, 128), dtype=np.uint16) & np.uint16(0x3FFF)
+    Kp = rng.integers(0, 2 ** 16, size=(n_pages, 2, P, 128), dtype=np.uint16)  # garbage where unused
+    Vp = rng.integers(0, 2 ** 16, size=(n_pages, 2, P, 128), dtype=np.uint16) & np.uint16(0x3FFF)
     Kp &= np.uint16(0x3FFF)
-    Cp = rng.integers(0, 256, size=(n_pages, P, 2, 32), dtype=np.uint8)
+    Cp = rng.integers(0, 256, size=(n_pages, 2, P, 32), dtype=np.uint8)
     for b in range(3):
         for lp in range(max_pages):
             page = perm[b, lp]
-            Kp[page] = inp["K"][b, :, lp * P:(lp + 1) * P].transpose(1, 0, 2)
-            Vp[page] = inp["V"][b, :, lp * P:(lp + 1) * P].transpose(1, 0, 2)
-            Cp[page] = codes[b, :, lp * P:(lp + 1) * P].transpose(1, 0, 2)
+            Kp[page] = inp["K"][b, :, lp * P:(lp + 1) * P]
+            Vp[page] = inp["V"][b, :, lp * P:(lp + 1) * P]
+            Cp[page] = codes[b, :, lp * P:(lp + 1) * P]
     out_p, idx_p = orc.decode_step_paged(inp["q"], Kp, Vp, Cp, perm, lens, 20)
     out_c, idx_c, _ = orc.decode_step(inp["q"], inp["K"], inp["V"], codes, lens, 20)
     assert np.array_equal(idx_p, idx_c)
@@ -520,7 +520,50 @@ def test_paged_step_equals_the_contiguous_step(orc):
 def test_paged_step_rejects_a_bad_table(orc):
     w = synth.WORKLOADS[2].scaled(Hq=2, Hkv=2, Nmax=32)
     inp = synth.make_inputs(w)
-    Kp = np.zeros((2, 16, 2, 128), np.uint16)
-    Cp = np.zeros((2, 16, 2, 32), np.uint8)
+    Kp = np.zeros((2, 2, 16, 128), np.uint16)
+    Cp = np.zeros((2, 2, 16, 32), np.uint8)
     with pytest.raises(ValueError):
         orc.decode_step_paged(inp["q"], Kp, Kp, Cp, np.array([[0, 5]], np.int32), np.array([32], np.int32), 4)
+
+
+# ---- forced rows and group-shared selection together
+
+def test_general_step_reduces_to_the_specific_steps(orc):
+    w = synth.WORKLOADS[4].scaled(B=2, Hq=6, Hkv=2, Nmax=60, len_range=None, n_needles=2)
+    inp = synth.make_inputs(w)
+    codes = orc.encode(inp["K"])
+    lens = np.array([60, 23], dtype=np.int32)
+    args = (inp["q"], inp["K"], inp["V"], codes, lens)
+    o, i = orc.decode_step_general(*args, 12, 2, 5, group_shared=False)
+    o2, i2 = orc.decode_step_forced(*args, 12, 2, 5)
+    assert np.array_equal(i, i2) and np.abs(o - o2).max() < 1e-12
+    o, i = orc.decode_step_general(*args, 12, group_shared=True)
+    o2, i2 = orc.decode_step_group_shared(*args, 12)
+    assert np.array_equal(i, i2) and np.abs(o - o2).max() < 1e-12
+    o, i = orc.decode_step_general(*args, 12)
+    o2, i2, _ = orc.decode_step(*args, 12)
+    assert np.array_equal(i, i2) and np.abs(o - o2).max() < 1e-12
+
+
+def test_general_step_forced_and_shared_match_brute_force(orc):
+    # summed unpacked-field L1 over the group, forced rows ranked at -1, Python sorted()
+    w = synth.WORKLOADS[4].scaled(B=2, Hq=4, Hkv=2, Nmax=36, len_range=None, n_needles=2)
+    inp = synth.make_inputs(w)
+    codes = orc.encode(inp["K"])
+    lens = np.array([36, 11], dtype=np.int32)
+    n_sink, n_recent = 2, 3
+    for budget in (3, 5, 9):
+        out, idx = orc.decode_step_general(inp["q"], inp["K"], inp["V"], codes, lens, budget, n_sink, n_recent,
+                                           group_shared=True)
+        for b in range(2):
+            n = int(lens[b])
+            for h in range(2):
+                kf = unpack(codes[b, h, :n])
+                tot = sum(np.abs(kf - unpack(orc.encode(inp["q"][b, 2 * h + g]))).sum(axis=1) for g in range(2))
+                rank = [(-1 if (t < n_sink or t >= n - n_recent) else int(tot[t]), t) for t in range(n)]
+                want = [t for _, t in sorted(rank)][:min(budget, n)]
+                assert idx[b, h, :len(want)].tolist() == want
+                assert (idx[b, h, len(want):] == -1).all()
+                for g in range(2):
+                    ref = _dense_sdpa(inp["q"][b, 2 * h + g], inp["K"][b, h][want], inp["V"][b, h][want])
+                    assert np.abs(out[b, 2 * h + g] - ref).max() < 1e-12
