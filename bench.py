@@ -1,13 +1,15 @@
 """Throughput of the ADAMAS sparse decode path on B200.
 
-One step = one attention layer's decode for the whole batch of the 128K-context
-workload (batch 1, 32 heads, head dim 128, context 131072, budget 1024): one
-launch of adamas_decode_step_append, which encodes the appended token's key into
-the code cache, encodes the query, scores all 131072 cached tokens per head by L1
-distance, selects the top 1024 and runs exact attention over the kept rows.  Four layer buffers rotate so that the
-working set (8.5 GiB) is far larger than L2.
+One step = one attention layer's decode for the whole batch of a workload: one
+launch that encodes the appended token's key into the code cache, encodes the
+query, scores every cached token of every kv head by the L1 distance of the
+codes, selects the budget of best tokens and runs exact attention over their
+K/V rows.  The default workload is the 128K-context one (batch 1, 32 heads,
+head dim 128, context 131072, budget 1024, per-head selection); four layer
+buffers rotate so that the working set is far larger than L2.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+                    [--workload NAME] [--budget K] [--policy per_head|group_shared]
 
 Prints one JSON line.  --impl reference times the CPU oracle on a bounded sample
 of the same workload.  Under torchrun every rank runs its own independent copy of
@@ -37,8 +39,9 @@ from compressed_sparse_kv_fp32_b200 import accounting, synth  # noqa: E402
 
 METRIC = "decode steps/s and achieved HBM GB/s (% of B200 peak) at 128K ctx, budget 1024"
 UNIT = "decode steps/s"
-WORKLOAD_ID = 3
-BUDGET = 1024
+DEFAULT_WORKLOAD = "mha32_128k"
+DEFAULT_BUDGET = {"single_head_4k": 64, "mha32_32k": 1024, "mha32_128k": 1024, "gqa8x4_b8_32k": 256,
+                  "gqa8x3_1m": 1024}
 LAYERS = 4
 FALLBACK_HBM_GBS = 6650.0
 
@@ -53,7 +56,24 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=500)
     ap.add_argument("--layers", type=int, default=LAYERS,
                     help="rotating layer buffers (fewer only for profiling captures)")
-    return ap.parse_args()
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(DEFAULT_BUDGET))
+    ap.add_argument("--budget", type=int, default=None)
+    ap.add_argument("--policy", default="per_head", choices=["per_head", "group_shared"])
+    a = ap.parse_args()
+    if a.budget is None:
+        a.budget = DEFAULT_BUDGET[a.workload]
+    return a
+
+
+def workload_of(name):
+    return next(w for w in synth.WORKLOADS.values() if w.name == name)
+
+
+def metric_of(args, w):
+    if args.workload == DEFAULT_WORKLOAD and args.budget == 1024 and args.policy == "per_head":
+        return METRIC
+    return (f"decode steps/s and achieved HBM GB/s (% of B200 peak): {w.name}, context {w.Nmax}, "
+            f"budget {args.budget}, {args.policy.replace('_', '-')} selection")
 
 
 def source_hash() -> str:
@@ -131,48 +151,66 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- CPU oracle (baseline / reference arm)
-def oracle_sample(w, heads: int, min_seconds: float):
-    """Time the oracle's decode step on `heads` heads of the workload at full context."""
+def oracle_sample(w, budget: int, policy: str, max_heads: int, min_seconds: float):
+    """Time the oracle's decode step on a sample of the workload's (sequence, kv head)
+    pairs at their full length; the value is scaled to whole steps."""
     from oracle import oracle
 
-    K = np.stack([synth.head_kv(w, 0, h)[0] for h in range(heads)])[None]
-    V = np.stack([synth.head_kv(w, 0, h)[1] for h in range(heads)])[None]
-    q = synth.query(w, 1)[:, :heads]
     lens = synth.seq_lens(w)
-    codes = oracle.encode(K)
+    pairs = [(b, h) for b in range(w.B) for h in range(w.Hkv)][:max_heads]
     cores = os.cpu_count() or 1
+    by_b = {}
+    for b, h in pairs:
+        by_b.setdefault(b, []).append(h)
+    sub = []
+    for b, hs in by_b.items():
+        n = int(lens[b])
+        K = np.stack([synth.head_kv(w, b, h, rows=n)[0] for h in hs])[None]
+        V = np.stack([synth.head_kv(w, b, h, rows=n)[1] for h in hs])[None]
+        qh = [h * w.G + g for h in hs for g in range(w.G)]
+        q = synth.query(w, 1)[b:b + 1, qh]
+        sub.append((q, K, V, oracle.encode(K), np.array([n], np.int32), len(hs)))
     reps, t0 = 0, time.perf_counter()
     while True:
-        oracle.decode_step(q, K, V, codes, lens, BUDGET, nthreads=min(cores, heads))
+        for q, K, V, codes, ln, nh in sub:
+            if policy == "group_shared":
+                oracle.decode_step_group_shared(q, K, V, codes, ln, budget)
+            else:
+                oracle.decode_step(q, K, V, codes, ln, budget, nthreads=min(cores, nh * w.G))
         reps += 1
         el = time.perf_counter() - t0
         if el >= min_seconds:
             break
-    steps = reps * heads / w.Hq
-    return {"value": steps / el, "unit": UNIT, "cores": min(cores, heads), "kind": "oracle",
-            "sample": f"{reps} oracle decode steps over {heads} of {w.Hq} heads at context {w.Nmax}, "
-                      f"budget {BUDGET} (query encode + L1 over every token + sort + float64 attention); "
-                      f"value scaled to whole {w.Hq}-head steps"}
+    steps = reps * len(pairs) / (w.B * w.Hkv)
+    used = 1 if policy == "group_shared" else min(cores, max(nh for *_, nh in sub) * w.G)
+    return {"value": steps / el, "unit": UNIT, "cores": used, "kind": "oracle",
+            "sample": f"{reps} oracle decode steps over {len(pairs)} of {w.B * w.Hkv} (sequence, kv head) pairs "
+                      f"at full length ({w.name}, budget {budget}, {policy.replace('_', '-')} selection: query "
+                      f"encode + L1 over every token + sort + float64 attention); value scaled to whole steps"}
 
 
-def config_block(w, n_layers=LAYERS):
-    return {"workload": f"{w.name}: batch {w.B}, {w.Hq} heads (MHA), head_dim {w.d}, context {w.Nmax}, "
-                        f"budget {BUDGET}, 1 appended token per step",
-            "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "context": w.Nmax, "budget": BUDGET, "head_dim": w.d,
+def config_block(w, args, n_layers=LAYERS):
+    lens = synth.seq_lens(w)
+    shape = (f"batch {w.B}, {w.Hq} query heads over {w.Hkv} kv heads, head_dim {w.d}, context {w.Nmax}"
+             + ("" if w.len_range is None else f" (lengths {int(lens.min())}..{int(lens.max())})"))
+    return {"workload": f"{w.name}: {shape}, budget {args.budget}, {args.policy.replace('_', '-')} selection, "
+                        f"1 appended token per sequence per step",
+            "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "context": w.Nmax, "budget": args.budget, "head_dim": w.d,
+            "policy": args.policy,
             "l2": f"{n_layers} rotating layer buffers (K, V, codes), working set "
-                  f"{n_layers * (2 * w.Hkv * w.Nmax * 256 + w.Hkv * w.Nmax * 32) / 2**30:.1f} GiB > L2",
+                  f"{n_layers * (2 * w.B * w.Hkv * w.Nmax * 256 + w.B * w.Hkv * w.Nmax * 32) / 2**30:.1f} GiB > L2",
             "parallelism": "independent replica per GPU"}
 
 
 def run_reference(args, rank, world):
-    w = synth.WORKLOADS[WORKLOAD_ID]
-    if rank != 0:
+    if rank != 0:  # rank 0 alone times the oracle and prints; the others do no work
         return
-    cb = oracle_sample(w, heads=min(8, os.cpu_count() or 1), min_seconds=15.0)
-    line = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": UNIT, "n_gpus": world,
+    w = workload_of(args.workload)
+    cb = oracle_sample(w, args.budget, args.policy, max_heads=min(8, os.cpu_count() or 1), min_seconds=15.0)
+    line = {"impl": "reference", "metric": metric_of(args, w), "value": cb["value"], "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 / cb["value"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u8/f64",
-            "data": "synthetic", "config": config_block(w), "cpu_baseline": cb,
+            "data": "synthetic", "config": config_block(w, args), "cpu_baseline": cb,
             "e2e": {"value": cb["value"], "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -205,33 +243,40 @@ def run_gpu(args, rank, world):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     lib = adamas.load()
-    w = synth.WORKLOADS[WORKLOAD_ID]
+    w = workload_of(args.workload)
     B, Hq, Hkv, N, d = w.B, w.Hq, w.Hkv, w.Nmax, w.d
-    ctx = N
-
-    # one layer generated on the host, copied into LAYERS device buffers
-    K_host = np.empty((B, Hkv, N, d), dtype=np.uint16)
-    V_host = np.empty_like(K_host)
-    for h in range(Hkv):
-        K_host[0, h], V_host[0, h] = synth.head_kv(w, 0, h)
+    budget = args.budget
+    shared = args.policy == "group_shared"
+    lens_np = synth.seq_lens(w)
 
     def to_dev(a):
-        return torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(torch.bfloat16)
 
+    # one layer generated on the host head by head, copied into every layer buffer
     n_layers = max(1, args.layers)
+    Ks = [torch.empty((B, Hkv, N, d), dtype=torch.bfloat16, device=dev) for _ in range(n_layers)]
+    Vs = [torch.empty_like(Ks[0]) for _ in range(n_layers)]
+    new_k = np.empty((B, Hkv, d), np.uint16)
+    new_v = np.empty_like(new_k)
+    for b in range(B):
+        for h in range(Hkv):
+            k, v = synth.head_kv(w, b, h)
+            kd, vd = to_dev(k), to_dev(v)
+            for l in range(n_layers):
+                Ks[l][b, h].copy_(kd)
+                Vs[l][b, h].copy_(vd)
+            new_k[b, h], new_v[b, h] = k[lens_np[b] - 1], v[lens_np[b] - 1]
     layers = []
     for l in range(n_layers):
-        K = to_dev(K_host)
-        V = to_dev(V_host)
         codes = torch.empty((B, Hkv, N, 32), dtype=torch.uint8, device=dev)
-        adamas.encode_keys(K, codes)
+        adamas.encode_keys(Ks[l], codes)
         q = to_dev(synth.query(w, l + 1))
         out = torch.empty((B, Hq, d), dtype=torch.float32, device=dev)
-        idx = torch.empty((B, Hq, BUDGET), dtype=torch.int32, device=dev)
-        ws = adamas.Workspace(B, Hq, Hkv, N, BUDGET, device=dev)
-        layers.append(dict(K=K, V=V, codes=codes, q=q, out=out, idx=idx, ws=ws))
-    lens = torch.full((B,), ctx, dtype=torch.int32, device=dev)
-    pos = torch.full((B,), ctx - 1, dtype=torch.int32, device=dev)   # the appended token's slot
+        idx = torch.empty((B, Hkv if shared else Hq, budget), dtype=torch.int32, device=dev)
+        ws = adamas.Workspace(B, Hq, Hkv, N, budget, device=dev)
+        layers.append(dict(K=Ks[l], V=Vs[l], codes=codes, q=q, out=out, idx=idx, ws=ws))
+    lens = torch.from_numpy(lens_np).to(dev)
+    pos = (lens - 1).to(torch.int32)   # the appended token: the newest of every sequence
     torch.cuda.synchronize()
 
     # ---- prefill encoder: the whole cache of one layer, the layers in turn (inputs > L2)
@@ -249,16 +294,20 @@ def run_gpu(args, rank, world):
     enc_us = g0.elapsed_time(g1) / enc_reps * 1e3
     (enc_us,) = max_over_ranks([enc_us], dev)
 
+    # one launch per step through the C ABI, arguments prepared once per layer
     stream = torch.cuda.current_stream().cuda_stream
-    calls = []
+    argss = []
     for L in layers:
-        calls.append((L["q"].data_ptr(), L["codes"].data_ptr(), L["K"].data_ptr(), L["V"].data_ptr(),
-                      lens.data_ptr(), pos.data_ptr(), B, Hq, Hkv, N, d, BUDGET, L["out"].data_ptr(),
-                      L["idx"].data_ptr(), L["ws"].buffer.data_ptr(), L["ws"].nbytes, stream))
-    f_step = lib.adamas_decode_step_append
+        argss.append(adamas.DecodeArgs(
+            L["q"].data_ptr(), L["codes"].data_ptr(), L["K"].data_ptr(), L["V"].data_ptr(), lens.data_ptr(),
+            B, Hq, Hkv, N, d, budget, L["out"].data_ptr(), L["idx"].data_ptr(), L["ws"].buffer.data_ptr(),
+            L["ws"].nbytes, pos.data_ptr(), None, None, None, 0, 0, 0, 0, 0,
+            adamas.SELECT_GROUP_SHARED if shared else adamas.SELECT_PER_HEAD))
+    refs = [ctypes.byref(a) for a in argss]
+    f_step = lib.adamas_decode_step_ex
 
     def step(i):
-        if f_step(*calls[i % n_layers]) != 0:
+        if f_step(refs[i % n_layers], stream) != 0:
             raise RuntimeError("decode step failed")
 
     gpu_id = "0"
@@ -307,33 +356,34 @@ def run_gpu(args, rank, world):
 
     elapsed_ms, dec_ms = max_over_ranks([elapsed_ms, dec_ms], dev)
 
-    # ---- end to end through the Python API: pinned host inputs in, results out, every step
+    # ---- end to end through the Python API: pinned host inputs in, results out, every
+    # step: one copy in (q and the new token's K and V rows), one launch (which writes
+    # the rows into the cache, encodes the key and decodes), one copy out (out and idx)
     e2e_steps = min(args.e2e_steps, K_steps)
-    # the step's inputs (q, new K row, new V row) travel in one pinned buffer and
-    # its results (out, idx) come back in one: one copy each way per step
     nq, nkv = B * Hq * d, B * Hkv * d
     in_pin = torch.empty(nq + 2 * nkv, dtype=torch.bfloat16).pin_memory()
     in_pin[:nq].copy_(torch.from_numpy(synth.query(w, 3).reshape(-1).view(np.int16)).view(torch.bfloat16))
-    in_pin[nq:nq + nkv].copy_(torch.from_numpy(K_host[:, :, ctx - 1].reshape(-1).view(np.int16)).view(torch.bfloat16))
-    in_pin[nq + nkv:].copy_(torch.from_numpy(V_host[:, :, ctx - 1].reshape(-1).view(np.int16)).view(torch.bfloat16))
+    in_pin[nq:nq + nkv].copy_(torch.from_numpy(new_k.reshape(-1).view(np.int16)).view(torch.bfloat16))
+    in_pin[nq + nkv:].copy_(torch.from_numpy(new_v.reshape(-1).view(np.int16)).view(torch.bfloat16))
     in_dev = torch.empty_like(in_pin, device=dev)
     q_dev = in_dev[:nq].view(B, Hq, d)
     krow_dev = in_dev[nq:nq + nkv].view(B, Hkv, d)
     vrow_dev = in_dev[nq + nkv:].view(B, Hkv, d)
-    n_out, n_idx = B * Hq * d, B * Hq * BUDGET   # fp32 and int32 words
+    rows = Hkv if shared else Hq
+    n_out, n_idx = B * Hq * d, B * rows * budget   # fp32 and int32 words
     res_dev = torch.empty(n_out + n_idx, dtype=torch.int32, device=dev)
     res_pin = torch.empty_like(res_dev, device="cpu").pin_memory()
     out_dev = res_dev[:n_out].view(torch.float32).view(B, Hq, d)
-    idx_dev = res_dev[n_out:].view(B, Hq, BUDGET)
+    idx_dev = res_dev[n_out:].view(B, rows, budget)
     h2d = in_pin.numel() * 2
     d2h = res_pin.numel() * 4
+    policy = adamas.SELECT_GROUP_SHARED if shared else adamas.SELECT_PER_HEAD
 
     def e2e_step(i):
         L = layers[i % n_layers]
         in_dev.copy_(in_pin, non_blocking=True)
-        L["K"][:, :, ctx - 1].copy_(krow_dev)
-        L["V"][:, :, ctx - 1].copy_(vrow_dev)
-        adamas.decode_step_append(q_dev, L["codes"], L["K"], L["V"], lens, pos, BUDGET, L["ws"], out_dev, idx_dev)
+        adamas.decode(q_dev, L["codes"], L["K"], L["V"], lens, budget, L["ws"], append_pos=pos, k_new=krow_dev,
+                      v_new=vrow_dev, policy=policy, out=out_dev, idx=idx_dev)
         res_pin.copy_(res_dev, non_blocking=True)
         torch.cuda.current_stream().synchronize()
 
@@ -354,27 +404,35 @@ def run_gpu(args, rank, world):
         return
     ms_per_step = elapsed_ms / K_steps
     value = job_value(world, K_steps, elapsed_ms)
-    step_bytes = accounting.decode_step_bytes([ctx] * B, Hq, Hkv, BUDGET, d)
+    keff = [min(budget, int(n)) for n in lens_np]
+    unique = sum(Hkv * k for k in keff) if shared else None
+    step_bytes = accounting.decode_step_bytes(lens_np, Hq, Hkv, budget, d, unique_rows=unique)
     enc_bytes = B * Hkv * accounting.encode_bytes_per_vector(d)
     peak, peak_kind = measured_peak()
     launch_bytes = step_bytes["total"] + enc_bytes   # the launch also encodes the appended keys
     achieved_dec = launch_bytes / (dec_ms / 1e3) / 1e9
     achieved_step = launch_bytes / (ms_per_step / 1e3) / 1e9
-    traffic = profiled_traffic("decode_step_kernel_mha32_128k")
+    headline = args.workload == DEFAULT_WORKLOAD and budget == 1024 and not shared
+    traffic = profiled_traffic("decode_step_kernel_mha32_128k") if headline else None
     enc_all = B * Hkv * N * accounting.encode_bytes_per_vector(d)
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K_steps,
+        "metric": metric_of(args, w), "value": value, "unit": UNIT, "n_gpus": world, "steps": K_steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "u8/fp32", "data": "synthetic",
-        "config": config_block(w, n_layers),
+        "config": config_block(w, args, n_layers),
         "achieved_hbm_gbs": achieved_step, "pct_of_peak_hbm": 100.0 * achieved_step / peak,
         "peak_hbm_gbs": peak, "peak_kind": peak_kind,
-        "roofline": {"bound": "hbm", "kernel": "decode_step_kernel", "achieved": achieved_dec, "peak": peak,
+        "roofline": {"bound": "hbm", "kernel": "decode_step_kernel" if not shared else "decode_step_ext_kernel",
+                     "achieved": achieved_dec, "peak": peak,
                      "unit": "GB/s", "frac": achieved_dec / peak, "traffic": traffic,
                      "algorithmic_bytes_per_launch": launch_bytes, "avg_launch_us": dec_ms * 1e3,
+                     "bytes": {"codes": step_bytes["codes"], "kv_rows": step_bytes["kv_rows"], "q": step_bytes["q"],
+                               "appended_keys": enc_bytes},
                      "peak_source": f"MEASURED_PEAKS.json hbm_gbs ({peak_kind})"},
         "e2e": ({"value": job_value(world, e2e_steps, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
-                 "d2h_bytes_per_step": d2h} if e2e_steps > 0 else None),
+                 "d2h_bytes_per_step": d2h,
+                 "per_step": "1 copy in, 1 launch (rows written, key encoded, decode), 1 copy out, 1 synchronise"}
+                if e2e_steps > 0 else None),
         "gpu_launches": K_steps,
         "clocks": clocks,
         "encode": {"kernel": "encode_keys_kernel", "what": f"prefill of {B * Hkv * N} key vectors ({N} tokens x "
@@ -384,7 +442,8 @@ def run_gpu(args, rank, world):
                    "frac": enc_all / (enc_us / 1e6) / 1e9 / peak},
     }
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = oracle_sample(w, heads=min(8, os.cpu_count() or 1), min_seconds=12.0)
+        line["cpu_baseline"] = oracle_sample(w, budget, args.policy, max_heads=min(8, os.cpu_count() or 1),
+                                             min_seconds=12.0)
     print(json.dumps(line), flush=True)
 
 
