@@ -31,6 +31,7 @@ SYMBOLS = (
     "adamas_status_string", "adamas_version", "adamas_last_error_string", "adamas_workspace_bytes", "adamas_workspace_init",
     "adamas_encode_keys", "adamas_decode_step", "adamas_score", "adamas_get_device_error",
     "adamas_decode_step_static", "adamas_decode_step_append", "adamas_decode_step_ex",
+    "adamas_debug_withhold_stage",
 )
 
 SELECT_PER_HEAD = 0
@@ -96,6 +97,8 @@ def load(path: str = LIBRARY) -> ctypes.CDLL:
         l.adamas_decode_step_append.restype = I
         l.adamas_decode_step_ex.argtypes = [ctypes.POINTER(DecodeArgs), P]
         l.adamas_decode_step_ex.restype = I
+        l.adamas_debug_withhold_stage.argtypes = [I]
+        l.adamas_debug_withhold_stage.restype = None
         _lib = l
         return l
 

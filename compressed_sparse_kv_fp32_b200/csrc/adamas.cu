@@ -8,6 +8,7 @@
 
 #include <cstdint>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "../../include/adamas.h"
@@ -526,10 +527,14 @@ static int check_decode_args(const adamas_decode_args& a, int64_t* Nmax_out) {
   return ADAMAS_OK;
 }
 
+// Test hook of adamas_debug_withhold_stage: the stage whose copy the next steps
+// never issue (-1: none).
+static std::atomic<int> g_withhold{-1};
+
 // The kernel instance a call needs: group-shared, general (any option), or plain.
 static int decode_mode(const adamas_decode_args& a) {
   if (a.policy == ADAMAS_SELECT_GROUP_SHARED) return kModeShared;
-  if (a.block_table || a.k_new || a.n_sink > 0 || a.n_recent > 0) return kModeGeneral;
+  if (a.block_table || a.k_new || a.n_sink > 0 || a.n_recent > 0 || g_withhold.load() >= 0) return kModeGeneral;
   return kModePlain;
 }
 
@@ -558,6 +563,7 @@ static int enqueue_decode(const adamas_decode_args& a, int64_t Nmax, unsigned ch
   prm.max_pages = a.block_table ? a.max_pages : 0;
   prm.n_sink = a.n_sink;
   prm.n_recent = a.n_recent;
+  prm.withhold = g_withhold.load();
   prm.B = a.B;
   prm.Hq = a.Hq;
   prm.Hkv = a.Hkv;
@@ -707,6 +713,8 @@ int adamas_decode_step_append(const void* q, uint8_t* codes, const void* K, cons
   a.append_pos = append_pos;
   return decode_with_workspace(a, (cudaStream_t)stream);
 }
+
+void adamas_debug_withhold_stage(int stage) { g_withhold.store(stage < 0 ? -1 : stage); }
 
 int adamas_decode_step_ex(const adamas_decode_args* args, adamas_stream_t stream) {
   if (!args) return ADAMAS_ERR_INVALID_ARG;

@@ -110,6 +110,35 @@ __device__ __forceinline__ void prefetch_l2(const void* p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(p) : "memory");
 }
 
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Wait for the phase with the given parity of `bar` to complete, for at most about
+// `limit_ns` nanoseconds of the global timer (checked every 128 polls; at most 2^26
+// polls in any case).  Returns false when it gives up.
+__device__ __forceinline__ bool mbar_wait_timed(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  const uint32_t a = smem_addr(bar);
+  uint64_t t_end = 0;
+  for (uint32_t i = 0; i < (1u << 26); ++i) {
+    uint32_t done;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(done)
+        : "r"(a), "r"(parity)
+        : "memory");
+    if (done) return true;
+    if ((i & 127u) == 127u) {
+      const uint64_t now = global_ns();
+      if (t_end == 0) t_end = now + limit_ns;
+      else if (now > t_end) return false;
+    }
+  }
+  return false;
+}
+
 // Bounded wait for the phase with the given parity of `bar` to complete.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t limit) {
   const uint32_t a = smem_addr(bar);

@@ -80,6 +80,7 @@ constexpr int kGatherBatch = 2 * kWorkerWarps * kGatherRows;  // rows per gather
 constexpr int kPushHistMax = 8;                       // C * G up to which histograms are pushed to peers
 constexpr uint32_t kPosMask = (1u << 23) - 1u;        // token offset within a block (list entries: d << 23 | t)
 constexpr uint32_t kWaitLimit = 1u << 20;             // mbarrier polls (about a second)
+constexpr uint64_t kWaitNs = 1000000000ull;          // time bound of a wait of the step with options
 
 struct DecodeParams {
   const uint16_t* q;
@@ -101,6 +102,7 @@ struct DecodeParams {
   int64_t n_pages;        // physical pages (paged cache)
   int page_size, max_pages;
   int n_sink, n_recent;   // forced rows: the first n_sink and the last n_recent tokens of each sequence
+  int withhold;           // test hook: the stage whose copy is never issued (-1: none)
   int B, Hq, Hkv;
   int64_t Nmax;           // tokens per sequence the cache can hold (paged: max_pages * page_size)
   int budget;

@@ -136,11 +136,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_ext_kernel(const Deco
       const int buf = i % NS;
       const int r0 = i * kStageRows, nr = min(kStageRows, seg_len - r0);
       if (lane == 0) {
-        if (i >= NS && !mbar_wait(&sm_empty[buf], (uint32_t)((i / NS) - 1) & 1u, kWaitLimit))
+        if (i >= NS && !mbar_wait_timed(&sm_empty[buf], (uint32_t)((i / NS) - 1) & 1u, kWaitNs))
           atomicOr(p.err, kErrTimeout);
-        mbar_arrive_expect_tx(&sm_full[buf], (uint32_t)nr * kCodeBytes);
+        if (i != p.withhold) mbar_arrive_expect_tx(&sm_full[buf], (uint32_t)nr * kCodeBytes);
       }
       __syncwarp();
+      if (i == p.withhold) return;  // test hook: this stage never arrives
       unsigned char* dst = ring + (size_t)buf * kStageBytes;
       const int64_t ta = t0 + r0, tb = ta + nr, P = p.page_size;
       for (int64_t lp = ta / P + lane; lp <= (tb - 1) / P; lp += 32) {
@@ -154,8 +155,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_ext_kernel(const Deco
         for (int i = 0; i < nst; ++i) {
           const int buf = i % NS;
           const int r0 = i * kStageRows, nr = min(kStageRows, seg_len - r0);
-          if (i >= NS && !mbar_wait(&sm_empty[buf], (uint32_t)((i / NS) - 1) & 1u, kWaitLimit))
+          if (i >= NS && !mbar_wait_timed(&sm_empty[buf], (uint32_t)((i / NS) - 1) & 1u, kWaitNs))
             atomicOr(p.err, kErrTimeout);
+          if (i == p.withhold) continue;  // test hook: this stage never arrives
           mbar_arrive_expect_tx(&sm_full[buf], (uint32_t)nr * kCodeBytes);
           bulk_copy_g2s(ring + (size_t)buf * kStageBytes, p.codes + (kv_base + t0 + r0) * kCodeBytes,
                         (uint32_t)nr * kCodeBytes, &sm_full[buf]);
@@ -203,7 +205,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_ext_kernel(const Deco
     }
     for (int i = 0; i < nst; ++i) {
       const int buf = i % NS;
-      if (!mbar_wait(&sm_full[buf], (uint32_t)(i / NS) & 1u, kWaitLimit)) atomicOr(p.err, kErrTimeout);
+      if (!mbar_wait_timed(&sm_full[buf], (uint32_t)(i / NS) & 1u, kWaitNs)) atomicOr(p.err, kErrTimeout);
       const int rows = min(kStageRows, seg_len - i * kStageRows);
       const unsigned char* st = ring + (size_t)buf * kStageBytes;
       uint4 kx[kRowsPerThread][2];

@@ -270,6 +270,16 @@ typedef struct adamas_decode_args {
 int adamas_decode_step_ex(const adamas_decode_args *args, adamas_stream_t stream);
 
 /*
+ * Test hook (not for production use): from now on every decode step runs its
+ * general kernel and never issues the bulk copy of code stage `stage` in any
+ * block, so the workers' bounded wait for that stage gives up after about a
+ * second, sets ADAMAS_DEVERR_TIMEOUT and the step completes with invalid outputs;
+ * no copy is left in flight.  A negative `stage` turns the hook off.  Process-wide
+ * and not thread-safe: for the tests of the timeout path only.
+ */
+void adamas_debug_withhold_stage(int stage);
+
+/*
  * Synchronise `stream`, then copy the workspace's device error word into
  * *error_word (ADAMAS_DEVERR_* bits).  Returns ADAMAS_OK when the word is zero,
  * ADAMAS_ERR_DEVICE when it is not.
