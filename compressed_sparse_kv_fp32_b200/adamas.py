@@ -31,7 +31,8 @@ SYMBOLS = (
     "adamas_status_string", "adamas_version", "adamas_last_error_string", "adamas_workspace_bytes", "adamas_workspace_init",
     "adamas_encode_keys", "adamas_decode_step", "adamas_score", "adamas_get_device_error",
     "adamas_decode_step_static", "adamas_decode_step_append", "adamas_decode_step_ex",
-    "adamas_debug_withhold_stage",
+    "adamas_static_device_error", "adamas_debug_withhold_stage",
+    "adamas_shard_workspace_bytes", "adamas_shard_score", "adamas_shard_attend", "adamas_merge_partials",
 )
 
 SELECT_PER_HEAD = 0
@@ -97,6 +98,16 @@ def load(path: str = LIBRARY) -> ctypes.CDLL:
         l.adamas_decode_step_append.restype = I
         l.adamas_decode_step_ex.argtypes = [ctypes.POINTER(DecodeArgs), P]
         l.adamas_decode_step_ex.restype = I
+        l.adamas_static_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32), P]
+        l.adamas_static_device_error.restype = I
+        l.adamas_shard_workspace_bytes.argtypes = [I, I, I, I64, I, I]
+        l.adamas_shard_workspace_bytes.restype = SZ
+        l.adamas_shard_score.argtypes = [P, P, P, I, I, I, I64, I, I, P, P, SZ, P]
+        l.adamas_shard_score.restype = I
+        l.adamas_shard_attend.argtypes = [P, P, P, P, I, I, I, I64, I, I, P, I, I, P, P, P, SZ, P]
+        l.adamas_shard_attend.restype = I
+        l.adamas_merge_partials.argtypes = [P, I, I, I, P, P]
+        l.adamas_merge_partials.restype = I
         l.adamas_debug_withhold_stage.argtypes = [I]
         l.adamas_debug_withhold_stage.restype = None
         _lib = l
@@ -141,12 +152,20 @@ def workspace_bytes(B: int, Hq: int, Hkv: int, Nmax: int, budget: int, d: int = 
     return int(n)
 
 
+def shard_workspace_bytes(B: int, Hq: int, Hkv: int, Nmax: int, budget: int, d: int = HEAD_DIM) -> int:
+    n = load().adamas_shard_workspace_bytes(B, Hq, Hkv, Nmax, d, budget)
+    if n == 0:
+        raise AdamasError(-2, "adamas_shard_workspace_bytes")
+    return int(n)
+
+
 class Workspace:
-    """Device workspace of adamas_decode_step, zero-filled on creation."""
+    """Device workspace of adamas_decode_step (or, with sharded=True, of the
+    sequence-sharded step's two halves), zero-filled on creation."""
 
     def __init__(self, B: int, Hq: int, Hkv: int, Nmax: int, budget: int, device=None,
-                 stream: Optional[torch.cuda.Stream] = None):
-        self.nbytes = workspace_bytes(B, Hq, Hkv, Nmax, budget)
+                 stream: Optional[torch.cuda.Stream] = None, sharded: bool = False):
+        self.nbytes = (shard_workspace_bytes if sharded else workspace_bytes)(B, Hq, Hkv, Nmax, budget)
         self.buffer = torch.empty(self.nbytes, dtype=torch.uint8,
                                   device=device if device is not None else "cuda")
         self.reset(stream)
@@ -309,3 +328,77 @@ def decode(q: torch.Tensor, codes: torch.Tensor, K: torch.Tensor, V: torch.Tenso
                    _ptr(block_table), n_pages, page_size, max_pages, n_sink, n_recent, policy)
     _check(load().adamas_decode_step_ex(ctypes.byref(a), _stream(stream)), "adamas_decode_step_ex")
     return out, idx
+
+
+# ---------------------------------------------------------------- sequence-sharded step
+HIST_STRIDE = 388      # ADAMAS_HIST_STRIDE: uint32 bins per (b, query head) of an exchanged histogram
+PARTIAL_FLOATS = 132   # ADAMAS_PARTIAL_FLOATS: fp32 per (b, query head) of a softmax state
+
+
+def _shard_shapes(q, codes_or_K, seq_lens):
+    _need(q, "q", torch.bfloat16)
+    if q.dim() != 3:
+        raise ValueError("q must be [B, Hq, 128]")
+    B, Hq, d = q.shape
+    if codes_or_K.dim() != 4:
+        raise ValueError("the cache must be [B, Hkv, Nmax, ...]")
+    _, Hkv, Nmax, _ = codes_or_K.shape
+    _need(seq_lens, "seq_lens", torch.int32, (B,))
+    return B, Hq, Hkv, Nmax, d
+
+
+def shard_score(q: torch.Tensor, codes: torch.Tensor, seq_lens: torch.Tensor, budget: int, workspace: Workspace,
+                hist: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """First half of the sharded step on this GPU's slice: returns its histograms
+    [B, Hq, HIST_STRIDE] int32 (uint32 counts), to be all-gathered in rank order."""
+    B, Hq, Hkv, Nmax, d = _shard_shapes(q, codes, seq_lens)
+    _need(codes, "codes", torch.uint8, (B, Hkv, Nmax, d // 4))
+    if hist is None:
+        hist = torch.empty((B, Hq, HIST_STRIDE), dtype=torch.int32, device=q.device)
+    _need(hist, "hist", torch.int32, (B, Hq, HIST_STRIDE))
+    _check(load().adamas_shard_score(q.data_ptr(), codes.data_ptr(), seq_lens.data_ptr(), B, Hq, Hkv, Nmax, d,
+                                     budget, hist.data_ptr(), workspace.buffer.data_ptr(), workspace.nbytes,
+                                     _stream(stream)), "adamas_shard_score")
+    return hist
+
+
+def shard_attend(q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, seq_lens: torch.Tensor, budget: int,
+                 hist_all: torch.Tensor, rank: int, workspace: Workspace, partial: Optional[torch.Tensor] = None,
+                 idx: Optional[torch.Tensor] = None,
+                 stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Second half on this GPU's slice, with hist_all [world, B, Hq, HIST_STRIDE] of
+    every slice: returns (partial [B, Hq, PARTIAL_FLOATS] fp32, idx [B, Hq, budget]
+    int32 holding the global indices of this slice's kept tokens, -1 elsewhere)."""
+    B, Hq, Hkv, Nmax, d = _shard_shapes(q, K, seq_lens)
+    _need(K, "K", torch.bfloat16, (B, Hkv, Nmax, d))
+    _need(V, "V", torch.bfloat16, (B, Hkv, Nmax, d))
+    if hist_all.dim() != 4:
+        raise ValueError("hist_all must be [world, B, Hq, HIST_STRIDE]")
+    world = hist_all.shape[0]
+    _need(hist_all, "hist_all", torch.int32, (world, B, Hq, HIST_STRIDE))
+    if partial is None:
+        partial = torch.empty((B, Hq, PARTIAL_FLOATS), dtype=torch.float32, device=q.device)
+    if idx is None:
+        idx = torch.empty((B, Hq, budget), dtype=torch.int32, device=q.device)
+    _need(partial, "partial", torch.float32, (B, Hq, PARTIAL_FLOATS))
+    _need(idx, "idx", torch.int32, (B, Hq, budget))
+    _check(load().adamas_shard_attend(q.data_ptr(), K.data_ptr(), V.data_ptr(), seq_lens.data_ptr(), B, Hq, Hkv,
+                                      Nmax, d, budget, hist_all.data_ptr(), world, int(rank), partial.data_ptr(),
+                                      idx.data_ptr() if budget > 0 else None, workspace.buffer.data_ptr(),
+                                      workspace.nbytes, _stream(stream)), "adamas_shard_attend")
+    return partial, idx
+
+
+def merge_partials(partials: torch.Tensor, out: Optional[torch.Tensor] = None,
+                   stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Attention output [B, Hq, 128] fp32 from the states [n, B, Hq, PARTIAL_FLOATS] of n slices."""
+    if partials.dim() != 4:
+        raise ValueError("partials must be [n, B, Hq, PARTIAL_FLOATS]")
+    n, B, Hq, _ = partials.shape
+    _need(partials, "partials", torch.float32, (n, B, Hq, PARTIAL_FLOATS))
+    if out is None:
+        out = torch.empty((B, Hq, HEAD_DIM), dtype=torch.float32, device=partials.device)
+    _need(out, "out", torch.float32, (B, Hq, HEAD_DIM))
+    _check(load().adamas_merge_partials(partials.data_ptr(), n, B, Hq, out.data_ptr(), _stream(stream)),
+           "adamas_merge_partials")
+    return out

@@ -199,6 +199,32 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(const uint16_t* __
   }
 }
 
+// ------------------------------------------------------------------ merge of softmax states
+// Combines n partial softmax states of every (b, query head) -- the slices of a
+// sharded sequence -- into the attention output.  A state is (m, l, -, -, o[128]):
+// m the largest scaled score of its kept tokens in log2 units (score / sqrt(128) *
+// log2 e), l the sum of 2^(s - m), o the 2^(s - m)-weighted sum of the V rows; a
+// state with m = -inf kept no token.  out = sum_r 2^(m_r - M) o_r / sum_r 2^(m_r - M) l_r
+// with M = max_r m_r (0 when no state kept a token).  One block per (b, query head),
+// one thread per output dimension.
+__global__ void __launch_bounds__(kDim) merge_partials_kernel(const float* __restrict__ part, int n, int64_t rows,
+                                                              float* __restrict__ out) {
+  const int64_t row = blockIdx.x;
+  const int e = threadIdx.x;
+  float M = -INFINITY;
+  for (int r = 0; r < n; ++r) M = fmaxf(M, part[((int64_t)r * rows + row) * kPartial]);
+  float L = 0.0f, O = 0.0f;
+  if (M != -INFINITY)
+    for (int r = 0; r < n; ++r) {
+      const float* st = part + ((int64_t)r * rows + row) * kPartial;
+      if (st[0] == -INFINITY) continue;
+      const float w = exp2f(st[0] - M);
+      L += st[1] * w;
+      O += st[4 + e] * w;
+    }
+  out[row * kDim + e] = M == -INFINITY ? 0.0f : O / L;
+}
+
 // ------------------------------------------------------------------ host side
 constexpr int kMaxDevices = 64;
 constexpr int kMinTokensPerBlock = 2048;  // fewer tokens per block than this only when the context is short
@@ -216,7 +242,7 @@ struct Plan;
 struct DeviceInfo {
   int sms = 0;
   size_t smem_optin = 0;
-  bool attrs_set[3][2][kMaxGroup + 1] = {};  // [mode][smem_d][G]
+  bool attrs_set[5][2][kMaxGroup + 1] = {};  // [mode][smem_d][G]
   OccEntry occ[kOccCache] = {};
   int n_occ = 0;
   int enc_blocks_per_sm = 0;  // resident prefill-encoder blocks per SM (0: not yet set up)
@@ -363,7 +389,7 @@ struct Plan {
   int dstride = 64;
   bool smem_d = true;
   size_t smem = 0;
-  size_t ctrl = 0, dspill = 0, total = 0;  // workspace offsets / size
+  size_t ctrl = 0, dspill = 0, bhist = 0, total = 0;  // workspace offsets / size
 };
 
 static size_t align256(size_t x) { return (x + 255) / 256 * 256; }
@@ -378,14 +404,15 @@ static int check_shape(int B, int Hq, int Hkv, int64_t Nmax, int d, int budget) 
 }
 
 // Shared-memory layout for `cluster` blocks per head: distances in shared memory
-// with as many ring stages as fit, else in the workspace with a full ring.
-static bool layout_for(int G, int64_t Nmax, int cluster, size_t optin, Plan* P) {
+// with as many ring stages as fit, else (or when `global_d`) in the workspace with
+// a full ring.
+static bool layout_for(int G, int64_t Nmax, int cluster, size_t optin, bool global_d, Plan* P) {
   const int64_t seg_cap = (Nmax + cluster - 1) / cluster;  // tokens of any block
   if (seg_cap >= (int64_t(1) << 23)) return false;          // token offsets are packed in 23 bits
   P->cluster = cluster;
   P->dstride = (int)((seg_cap < 1 ? 1 : seg_cap) + 63) / 64 * 64;
   bool found = false;
-  for (int pass = 0; pass < 2 && !found; ++pass) {
+  for (int pass = global_d ? 1 : 0; pass < 2 && !found; ++pass) {
     const bool in_smem = pass == 0;
     for (int ns = kMaxStages; ns >= kMinStages && !found; --ns) {
       const size_t s = DecodeSmem::total(G, cluster, ns, P->dstride, in_smem);
@@ -406,6 +433,7 @@ static bool layout_for(int G, int64_t Nmax, int cluster, size_t optin, Plan* P) 
 // tokens per block; 1 when even single blocks need several waves.
 static int make_plan_uncached(int B, int Hq, int Hkv, int64_t Nmax, int mode, DeviceInfo& dev, Plan* P) {
   const int G = Hq / Hkv;
+  const bool sharded = mode == kModeShardScore || mode == kModeShardAttend;
   const int heads = B * Hkv;
   P->G = G;
   int want = heads > 0 ? dev.sms / heads : 1;
@@ -416,7 +444,7 @@ static int make_plan_uncached(int B, int Hq, int Hkv, int64_t Nmax, int mode, De
   bool found = false;
   for (int c = want; c >= 1 && !found; --c) {
     Plan t = *P;
-    if (!layout_for(G, Nmax, c, dev.smem_optin, &t)) continue;
+    if (!layout_for(G, Nmax, c, dev.smem_optin, sharded, &t)) continue;
     const void* fn = decode_fn_for(G, t.smem_d, mode);
     int rc = kernel_attrs(dev, fn, G, t.smem_d, mode);
     if (rc != ADAMAS_OK) return rc;
@@ -433,6 +461,8 @@ static int make_plan_uncached(int B, int Hq, int Hkv, int64_t Nmax, int mode, De
   P->ctrl = off;   off += align256(64 * sizeof(uint32_t));
   P->dspill = off;
   off += P->smem_d ? 0 : align256((size_t)P->grid * G * P->dstride * sizeof(uint16_t));
+  P->bhist = off;  // the sharded step's per-block histograms (kept between its two launches)
+  off += sharded ? align256((size_t)P->grid * G * kHistStride * sizeof(uint32_t)) : 0;
   P->total = off;
   return ADAMAS_OK;
 }
@@ -721,6 +751,117 @@ int adamas_decode_step_ex(const adamas_decode_args* args, adamas_stream_t stream
   return decode_with_workspace(*args, (cudaStream_t)stream);
 }
 
+// ------------------------------------------------------------------ sequence-sharded step
+static_assert(kHistStride == ADAMAS_HIST_STRIDE && kPartial == ADAMAS_PARTIAL_FLOATS,
+              "the exchange layouts of the header");
+// Both halves use one plan (the score half's), so that block i of the attend half
+// finds the distances and histograms that block i of the score half left.
+static int shard_plan(int B, int Hq, int Hkv, int64_t Nmax, int d, int budget, Plan* P) {
+  int rc = check_shape(B, Hq, Hkv, Nmax, d, budget);
+  if (rc != ADAMAS_OK) return rc;
+  DeviceInfo* dev = nullptr;
+  int devno = 0;
+  if ((rc = device_info(&dev, &devno)) != ADAMAS_OK) return rc;
+  if ((rc = make_plan(B, Hq, Hkv, Nmax, kModeShardScore, *dev, devno, P)) != ADAMAS_OK) return rc;
+  // the attend half's instance: the same shared memory and cluster shape
+  const void* fn = decode_fn_for(P->G, false, kModeShardAttend);
+  if ((rc = kernel_attrs(*dev, fn, P->G, false, kModeShardAttend)) != ADAMAS_OK) return rc;
+  int n = 0;
+  if ((rc = active_clusters(*dev, fn, P->cluster, P->smem, &n)) != ADAMAS_OK) return rc;
+  return n >= 1 ? ADAMAS_OK : ADAMAS_ERR_UNSUPPORTED;
+}
+
+static void shard_params(DecodeParams& prm, const Plan& P, unsigned char* ws, const void* q, const int32_t* seq_lens,
+                         int B, int Hq, int Hkv, int64_t Nmax, int budget) {
+  prm.q = static_cast<const uint16_t*>(q);
+  prm.seq_lens = seq_lens;
+  prm.err = reinterpret_cast<uint32_t*>(ws + P.ctrl) + 2;
+  prm.dglobal = reinterpret_cast<uint16_t*>(ws + P.dspill);
+  prm.blk_hist = reinterpret_cast<uint32_t*>(ws + P.bhist);
+  prm.withhold = -1;
+  prm.page_size = 1;
+  prm.B = B;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.Nmax = Nmax;
+  prm.budget = budget;
+  prm.cluster = P.cluster;
+  prm.nstages = P.nstages;
+  prm.dstride = P.dstride;
+  prm.shard_world = 1;
+}
+
+size_t adamas_shard_workspace_bytes(int B, int Hq, int Hkv, int64_t Nmax, int d, int budget) {
+  Plan P;
+  if (shard_plan(B, Hq, Hkv, Nmax, d, budget, &P) != ADAMAS_OK) return 0;
+  return P.total;
+}
+
+int adamas_shard_score(const void* q, const uint8_t* codes, const int32_t* seq_lens, int B, int Hq, int Hkv,
+                       int64_t Nmax, int d, int budget, uint32_t* hist, void* workspace, size_t workspace_bytes,
+                       adamas_stream_t stream) {
+  int rc = check_shape(B, Hq, Hkv, Nmax, d, budget);
+  if (rc != ADAMAS_OK || B == 0) return rc;
+  if (!q || !seq_lens || !hist || (Nmax > 0 && !codes)) return ADAMAS_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(codes, 32) || !aligned(seq_lens, 4) || !aligned(hist, 4))
+    return ADAMAS_ERR_INVALID_ARG;
+  Plan P;
+  if ((rc = shard_plan(B, Hq, Hkv, Nmax, d, budget, &P)) != ADAMAS_OK) return rc;
+  if (!workspace || workspace_bytes < P.total || !aligned(workspace, 16)) return ADAMAS_ERR_WORKSPACE;
+  cudaStream_t st = (cudaStream_t)stream;
+  const cudaError_t e = cudaMemsetAsync(hist, 0, (size_t)B * Hq * kHistStride * sizeof(uint32_t), st);
+  if (e != cudaSuccess) return cuda_fail(e);
+  DecodeParams prm = {};
+  shard_params(prm, P, static_cast<unsigned char*>(workspace), q, seq_lens, B, Hq, Hkv, Nmax, budget);
+  prm.codes = codes;
+  prm.shard_hist = hist;
+  return launch_decode(prm, P, kModeShardScore, st);
+}
+
+int adamas_shard_attend(const void* q, const void* K, const void* V, const int32_t* seq_lens, int B, int Hq, int Hkv,
+                        int64_t Nmax, int d, int budget, const uint32_t* hist_all, int world, int rank,
+                        float* partial, int32_t* idx, void* workspace, size_t workspace_bytes,
+                        adamas_stream_t stream) {
+  int rc = check_shape(B, Hq, Hkv, Nmax, d, budget);
+  if (rc != ADAMAS_OK || B == 0) return rc;
+  if (world < 1 || rank < 0 || rank >= world) return ADAMAS_ERR_INVALID_ARG;
+  if (!q || !seq_lens || !hist_all || !partial || (budget > 0 && !idx) || (Nmax > 0 && (!K || !V)))
+    return ADAMAS_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(seq_lens, 4) || !aligned(hist_all, 4) ||
+      !aligned(partial, 16) || !aligned(idx, 4))
+    return ADAMAS_ERR_INVALID_ARG;
+  Plan P;
+  if ((rc = shard_plan(B, Hq, Hkv, Nmax, d, budget, &P)) != ADAMAS_OK) return rc;
+  if (!workspace || workspace_bytes < P.total || !aligned(workspace, 16)) return ADAMAS_ERR_WORKSPACE;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (budget > 0) {  // slots of other slices' tokens and past k_eff stay -1
+    const cudaError_t e = cudaMemsetAsync(idx, 0xFF, (size_t)B * Hq * budget * sizeof(int32_t), st);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  DecodeParams prm = {};
+  shard_params(prm, P, static_cast<unsigned char*>(workspace), q, seq_lens, B, Hq, Hkv, Nmax, budget);
+  prm.K = static_cast<const uint16_t*>(K);
+  prm.V = static_cast<const uint16_t*>(V);
+  prm.idx = idx;
+  prm.hist_all = hist_all;
+  prm.partial = partial;
+  prm.shard_rank = rank;
+  prm.shard_world = world;
+  return launch_decode(prm, P, kModeShardAttend, st);
+}
+
+int adamas_merge_partials(const float* partials, int n, int B, int Hq, float* out, adamas_stream_t stream) {
+  if (n < 1 || B < 0 || Hq < 0) return ADAMAS_ERR_INVALID_ARG;
+  const int64_t rows = (int64_t)B * Hq;
+  if (rows == 0) return ADAMAS_OK;
+  if (rows > INT32_MAX) return ADAMAS_ERR_UNSUPPORTED;
+  if (!partials || !out || !aligned(partials, 16) || !aligned(out, 16)) return ADAMAS_ERR_INVALID_ARG;
+  merge_partials_kernel<<<(unsigned)rows, kDim, 0, (cudaStream_t)stream>>>(partials, n, rows, out);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e);
+  return ADAMAS_OK;
+}
+
 int adamas_score(const void* q, const uint8_t* codes, const int32_t* seq_lens, int B, int Hq, int Hkv, int64_t Nmax,
                  int d, uint16_t* dist, adamas_stream_t stream) {
   const int rc = check_shape(B, Hq, Hkv, Nmax, d, 0);
@@ -780,24 +921,59 @@ constexpr size_t kStaticScratchBytes = size_t(4) << 20;  // 4 MiB on every devic
 static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
 static std::mutex g_static_mutex;
-static void* g_static_scratch_ptr[kMaxDevices] = {};
 
-// Device address of g_static_scratch on the current device.  In host code the
-// array's name is only a host-side stand-in, so the address is looked up once
-// per device, with that device current, and cached.
-static int static_scratch(void** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+// Driver calls reached through the runtime's entry-point query (the library links
+// only the runtime): the current context and its process-unique id.
+typedef int (*CtxGetCurrentFn)(void** ctx);
+typedef int (*CtxGetIdFn)(void* ctx, unsigned long long* id);
+
+static int driver_fn(const char* name, void** fn) {
+  cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+  const cudaError_t e = cudaGetDriverEntryPointByVersion(name, fn, 12000, cudaEnableDefault, &q);
   if (e != cudaSuccess) return cuda_fail(e);
-  if (dev < 0 || dev >= kMaxDevices) return ADAMAS_ERR_UNSUPPORTED;
+  return q == cudaDriverEntryPointSuccess && *fn ? ADAMAS_OK : ADAMAS_ERR_UNSUPPORTED;
+}
+
+// Device address of g_static_scratch in the current context.  In host code the
+// array's name is only a host-side stand-in: the address is looked up with the
+// context current and cached under the context's id, which the driver never
+// reuses within a process.  A context created later (after cudaDeviceReset, or
+// another context made current) has another id and gets its own lookup, so a
+// cached address never outlives the context it was taken in.
+static int static_scratch(void** out) {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  constexpr int kSlots = 16;
+  static unsigned long long ids[kSlots] = {};
+  static void* ptrs[kSlots] = {};
+  static int next = 0;
   std::lock_guard<std::mutex> lock(g_static_mutex);
-  if (!g_static_scratch_ptr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_static_scratch);
+  int rc;
+  if (!get_current && (rc = driver_fn("cuCtxGetCurrent", reinterpret_cast<void**>(&get_current))) != ADAMAS_OK)
+    return rc;
+  if (!get_id && (rc = driver_fn("cuCtxGetId", reinterpret_cast<void**>(&get_id))) != ADAMAS_OK) return rc;
+  void* ctx = nullptr;
+  if (get_current(&ctx) != 0 || ctx == nullptr) {  // none yet: the runtime makes the device's primary context current
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaSetDevice(dev);
     if (e != cudaSuccess) return cuda_fail(e);
-    g_static_scratch_ptr[dev] = p;
+    if (get_current(&ctx) != 0 || ctx == nullptr) return ADAMAS_ERR_CUDA;
   }
-  *out = g_static_scratch_ptr[dev];
+  unsigned long long id = 0;
+  if (get_id(ctx, &id) != 0) return ADAMAS_ERR_CUDA;
+  for (int i = 0; i < kSlots; ++i)
+    if (ptrs[i] && ids[i] == id) {
+      *out = ptrs[i];
+      return ADAMAS_OK;
+    }
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
+  if (e != cudaSuccess) return cuda_fail(e);
+  ids[next] = id;
+  ptrs[next] = p;
+  next = (next + 1) % kSlots;
+  *out = p;
   return ADAMAS_OK;
 }
 
@@ -824,4 +1000,12 @@ extern "C" int adamas_decode_step_static(const void* q, const uint8_t* codes, co
   const cudaError_t e = cudaMemsetAsync(scratch, 0, P.dspill, st);
   if (e != cudaSuccess) return cuda_fail(e);
   return enqueue_decode(a, Nm, static_cast<unsigned char*>(scratch), P, st);
+}
+
+extern "C" int adamas_static_device_error(uint32_t* error_word, adamas_stream_t stream) {
+  if (!error_word) return ADAMAS_ERR_INVALID_ARG;
+  void* scratch = nullptr;
+  const int rc = adamas::static_scratch(&scratch);
+  if (rc != ADAMAS_OK) return rc;
+  return adamas_get_device_error(scratch, adamas::kStaticScratchBytes, error_word, stream);
 }

@@ -103,6 +103,12 @@ struct DecodeParams {
   int page_size, max_pages;
   int n_sink, n_recent;   // forced rows: the first n_sink and the last n_recent tokens of each sequence
   int withhold;           // test hook: the stage whose copy is never issued (-1: none)
+  // sequence-sharded step: the cache holds one contiguous slice of every sequence
+  uint32_t* shard_hist;       // score: [B][Hq][kHistStride] this slice's histograms (added into, zeroed first)
+  const uint32_t* hist_all;   // attend: [world][B][Hq][kHistStride] the histograms of every slice, in order
+  uint32_t* blk_hist;         // [grid][G][kHistStride] each block's own histograms (workspace)
+  float* partial;             // attend: [B][Hq][kPartial] this slice's softmax state (m, l, -, -, o[128])
+  int shard_rank, shard_world;
   int B, Hq, Hkv;
   int64_t Nmax;           // tokens per sequence the cache can hold (paged: max_pages * page_size)
   int budget;

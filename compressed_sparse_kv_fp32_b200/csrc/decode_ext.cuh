@@ -11,10 +11,24 @@ namespace adamas {
 
 // Kernel modes: the plain step has its own kernel (decode_plain.cuh); this one is
 // the general per-head step and the group-shared step, which read the options
-// (paged cache, forced rows, rows written by the launch) at run time.
+// (paged cache, forced rows, rows written by the launch) at run time, and the two
+// halves of the sequence-sharded step.
 constexpr int kModePlain = 0;
 constexpr int kModeGeneral = 1;
 constexpr int kModeShared = 2;
+// Sequence-sharded step: each GPU holds one contiguous slice of every sequence.
+//   kModeShardScore   phase 1 only: the slice's distances go to the workspace, each
+//                     block's histograms to the workspace and their sum over the
+//                     slice to the exchange buffer.
+//   kModeShardAttend  phase 2 and the merge, with the threshold and rank bases taken
+//                     from every slice's histograms (the exchange buffers of all
+//                     GPUs, gathered in slice order); the output is this slice's
+//                     softmax state, and idx holds the global indices of the
+//                     slice's kept tokens.
+// The histogram exchange makes the selection exactly the one of the whole
+// sequence: the slices play the part the blocks of a cluster play inside a GPU.
+constexpr int kModeShardScore = 3;
+constexpr int kModeShardAttend = 4;
 
 // SMEM_D: the block's distances live in shared memory (else in the workspace).
 // MODE kModeShared: group-shared selection -- the distances of the G query heads are
@@ -24,6 +38,9 @@ template <int G, bool SMEM_D, int MODE>
 __global__ void __launch_bounds__(kThreads, 1) decode_step_ext_kernel(const DecodeParams p) {
   constexpr bool SHARED = MODE == kModeShared;
   constexpr bool GENERAL = MODE != kModePlain;
+  constexpr bool SCORE_ONLY = MODE == kModeShardScore;
+  constexpr bool ATTEND_ONLY = MODE == kModeShardAttend;
+  static_assert(!(SCORE_ONLY || ATTEND_ONLY) || !SMEM_D, "the sharded step keeps its distances in the workspace");
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ __align__(8) uint64_t sm_full[kMaxStages];
   __shared__ __align__(8) uint64_t sm_empty[kMaxStages];
@@ -35,6 +52,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_ext_kernel(const Deco
   __shared__ long long sm_tmp[kWorkerWarps];
   __shared__ uint32_t sm_sink[32];  // per-lane target of the unused atomics of a batch
   __shared__ int sm_round[2];       // totals of one round of the ordered pass
+  __shared__ unsigned long long sm_len[2];  // sharded step: tokens of the sequence before this slice, in all
 
   cg::cluster_group cluster = cg::this_cluster();
   const int C = p.cluster;
@@ -83,7 +101,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_ext_kernel(const Deco
     if (rank == 0 && tid == 0) atomicOr(p.err, kErrSeqLen);
     len_b = len_b < 0 ? 0 : p.Nmax;
   }
-  const int keff = (int)min((int64_t)p.budget, len_b);
+  // k_eff of the sequence (of the whole sequence in the sharded step: set below)
+  int keff = (int)min((int64_t)p.budget, len_b);
   const bool forced = GENERAL && (p.n_sink > 0 || p.n_recent > 0);
   // distance bins: [0, 384] per query head, [0, 384 G] summed over a group; one more
   // when forced rows take bin 0
@@ -95,7 +114,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_ext_kernel(const Deco
     seg_len = p.dstride;
   }
   const int NS = p.nstages;
-  const int nst = keff > 0 ? (seg_len + kStageRows - 1) / kStageRows : 0;  // nothing to score without a budget
+  // nothing to score without a budget; the attend half of the sharded step scores nothing
+  const int nst = !ATTEND_ONLY && keff > 0 ? (seg_len + kStageRows - 1) / kStageRows : 0;
   const int64_t kv_base = (int64_t)hk * p.Nmax;
   // appended key of this (b, kv head): encoded by a spare worker warp of the block
   // that owns its position (the last block when it lies past the sequence) while
@@ -120,8 +140,41 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_ext_kernel(const Deco
   for (int i = tid; i < G * kHistStride; i += kThreads) sm_hist[i] = 0u;
   if (tid < kMaxGroup) sm_T[tid] = kBins - 1;  // always overwritten when the histograms are consistent
   if (tid < 2) sm_round[tid] = 0;  // a block without tokens runs no round of the ordered pass
+  if (tid < 2) sm_len[tid] = 0ull;
 
   __syncthreads();
+  // Sharded step: the sequence's length and this slice's first index are the
+  // histogram totals (every scored token is counted once per query head) of all
+  // slices and of the slices before this one.
+  int64_t ofs = 0;
+  if constexpr (ATTEND_ONLY) {
+    const uint32_t* h0 = p.hist_all + ((int64_t)b * p.Hq + (int64_t)kvh * G) * kHistStride;
+    const int64_t rs = (int64_t)p.B * p.Hq * kHistStride;
+    unsigned long long before = 0ull, total = 0ull;
+    for (int i = tid; i < p.shard_world * kBins; i += kThreads) {
+      const int r = i / kBins, d = i - r * kBins;
+      const uint32_t v = h0[r * rs + d];
+      total += v;
+      if (r < p.shard_rank) before += v;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      total += __shfl_xor_sync(0xffffffffu, total, o);
+      before += __shfl_xor_sync(0xffffffffu, before, o);
+    }
+    if (lane == 0) {
+      atomicAdd(&sm_len[0], before);
+      atomicAdd(&sm_len[1], total);
+    }
+    __syncthreads();
+    ofs = (int64_t)sm_len[0];
+    int64_t len_g = (int64_t)sm_len[1];
+    if (len_g > INT32_MAX) {  // global indices are int32
+      if (rank == 0 && tid == 0) atomicOr(p.err, kErrSeqLen);
+      len_g = INT32_MAX;
+    }
+    keff = (int)min((int64_t)p.budget, len_g);
+  }
   // Every block of the cluster has started (and may be written to through
   // distributed shared memory) once every thread has arrived here; each thread
   // waits on it before its first such access.
@@ -168,7 +221,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_ext_kernel(const Deco
     __syncwarp();
     cluster_wait();
   } else {
-    if (warp < G && keff > 0) {
+    if (!ATTEND_ONLY && warp < G && keff > 0) {
       const uint32_t w = encode128_warp(p.q + ((int64_t)b * p.Hq + kvh * G + warp) * kDim, lane);
       if (lane < kCodeWords) {
         sm_q[warp * kCodeWords + lane] = w;
@@ -284,7 +337,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_ext_kernel(const Deco
     }
 
     cluster_wait();
-    if (push_hist && keff > 0) {  // own histograms into every block's table (row `rank`)
+    if constexpr (SCORE_ONLY) {  // own histograms to the workspace, and into the slice's sums
+      worker_sync();
+      uint32_t* bh = p.blk_hist + (size_t)blockIdx.x * G * kHistStride;
+      for (int i = tid; i < G * kHistStride; i += kWorkers) {
+        const uint32_t v = sm_hist[i];
+        bh[i] = v;
+        const int g = i / kHistStride, d = i - g * kHistStride;
+        if (v != 0u) atomicAdd(p.shard_hist + ((int64_t)b * p.Hq + kvh * G + g) * kHistStride + d, v);
+      }
+    } else if constexpr (ATTEND_ONLY) {  // own histograms from the score half
+      const uint32_t* bh = p.blk_hist + (size_t)blockIdx.x * G * kHistStride;
+      for (int i = tid; i < G * kHistStride; i += kWorkers) sm_hist[i] = bh[i];
+    } else if (push_hist && keff > 0) {  // own histograms into every block's table (row `rank`)
       worker_sync();
       for (int r = 0; r < C; ++r) {
         uint32_t* tab = cluster.map_shared_rank(sm_htab, r) + (size_t)rank * G * kHistStride;
@@ -292,6 +357,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_ext_kernel(const Deco
       }
     }
   }
+  if constexpr (SCORE_ONLY) return;  // no peer reads this block's shared memory in this mode
   __syncthreads();
   cluster.sync();  // every block's histograms are complete and visible to the cluster
 
@@ -314,18 +380,36 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_ext_kernel(const Deco
         auto bin = [&](int d, long long& H, long long& P, long long& own) {
           H = P = own = 0;
           if (d >= nbins) return;
-          uint32_t v[kMaxCluster];
+          if constexpr (ATTEND_ONLY) {
+            // this slice: the blocks of the cluster; the other slices: their sums
+            const uint32_t* bh = p.blk_hist + ((size_t)hk * C * G + g) * kHistStride + d;
+            for (int r = 0; r < C; ++r) {
+              const uint32_t v = bh[(size_t)r * G * kHistStride];
+              H += v;
+              if (r < rank) P += v;
+            }
+            const uint32_t* ha = p.hist_all + ((int64_t)b * p.Hq + (int64_t)kvh * G + g) * kHistStride + d;
+            const int64_t rs = (int64_t)p.B * p.Hq * kHistStride;
+            for (int r = 0; r < p.shard_world; ++r) {
+              if (r == p.shard_rank) continue;
+              const uint32_t v = ha[r * rs];
+              H += v;
+              if (r < p.shard_rank) P += v;
+            }
+          } else {
+            uint32_t v[kMaxCluster];
 #pragma unroll
-          for (int r = 0; r < kMaxCluster; ++r) {
-            v[r] = 0u;
-            if (r < C)
-              v[r] = push_hist ? sm_htab[((size_t)r * G + g) * kHistStride + d]
-                               : cluster.map_shared_rank(sm_hist, r)[g * kHistStride + d];
-          }
+            for (int r = 0; r < kMaxCluster; ++r) {
+              v[r] = 0u;
+              if (r < C)
+                v[r] = push_hist ? sm_htab[((size_t)r * G + g) * kHistStride + d]
+                                 : cluster.map_shared_rank(sm_hist, r)[g * kHistStride + d];
+            }
 #pragma unroll
-          for (int r = 0; r < kMaxCluster; ++r) {
-            H += v[r];
-            if (r < rank) P += v[r];
+            for (int r = 0; r < kMaxCluster; ++r) {
+              H += v[r];
+              if (r < rank) P += v[r];
+            }
           }
           own = sm_hist[g * kHistStride + d];
         };
@@ -359,6 +443,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_ext_kernel(const Deco
     worker_sync();
 
     const int hw = tid >> 4, hl = tid & 15;  // two half-warps per worker warp
+    const int64_t it0 = t0 + ofs;  // index (in the whole sequence) of the block's first token
     const float kScoreScale = 0.08838834764831845f * 1.4426950408889634f;  // log2(e)/sqrt(128)
     // warp slices over 8-position groups of the block's distances (full scans)
     const int ngrp = (seg_len + 7) >> 3;
@@ -432,7 +517,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_ext_kernel(const Deco
           } else {
             if (at_eq < tie_quota && n_lt + at_eq < n_kept) {
               sm_kept[n_lt + at_eq] = (int32_t)pos;
-              idx_h[tie_base + at_eq] = (int32_t)(t0 + pos);
+              idx_h[tie_base + at_eq] = (int32_t)(it0 + pos);
             }
             ++at_eq;
           }
@@ -465,7 +550,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_ext_kernel(const Deco
         const uint64_t kk = sm_keys[i];
         const uint32_t d = (uint32_t)(kk >> 32);
         const uint32_t slot = rank_g[d] + ((uint32_t)i - lpre_g[d]);
-        if (slot < (uint32_t)keff) idx_h[slot] = (int32_t)(t0 + (uint32_t)kk);
+        if (slot < (uint32_t)keff) idx_h[slot] = (int32_t)(it0 + (uint32_t)kk);
       }
       worker_sync();
     };
@@ -619,7 +704,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_ext_kernel(const Deco
           for (; q < gn; ++q) r += ((uint32_t)grp_list[q] & kPosMask) < tpos;
           const int slot = (int)rank_g[d] + r;
           if (slot < keff) {
-            idx_h[slot] = (int32_t)(t0 + tpos);
+            idx_h[slot] = (int32_t)(it0 + tpos);
             sm_kept[gb + r] = (int32_t)tpos;
           }
         }
@@ -719,7 +804,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_ext_kernel(const Deco
                     if (r0 == 0 && (meq[it] & (1u << e))) {
                       const int tie = at_eq++;
                       if (tie < tie_quota) {
-                        if (c0 == 0) idx_h[tie_base + tie] = (int32_t)(t0 + pos);
+                        if (c0 == 0) idx_h[tie_base + tie] = (int32_t)(it0 + pos);
                         const int kp = n_lt + tie - c0;
                         if (kp >= 0 && kp < n_win) sm_kept[kp] = (int32_t)pos;
                       }
@@ -756,7 +841,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_ext_kernel(const Deco
                   if (w < warp) before += lds32(ca + w * kHistStride * 4);
                 before += (uint32_t)__popc(peers & lt);  // rank of the token among the block's equal distances
                 const uint32_t tpos = ent & kPosMask;
-                if (c0 == 0 && rank_g[d] + before < (uint32_t)keff) idx_h[rank_g[d] + before] = (int32_t)(t0 + tpos);
+                if (c0 == 0 && rank_g[d] + before < (uint32_t)keff) idx_h[rank_g[d] + before] = (int32_t)(it0 + tpos);
                 const int kp = (int)(lpre_g[d] + before) - c0;
                 if (kp >= 0 && kp < n_win) sm_kept[kp] = (int32_t)tpos;
               }
@@ -826,12 +911,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_ext_kernel(const Deco
     for (int g = rank; g < G; g += C) {
       const int64_t hq = (int64_t)b * p.Hq + kvh * G + g;
       for (int e = tid; e < kDim; e += kWorkers) {
-        float res = 0.0f;
+        float res = 0.0f, M = -INFINITY, L = 0.0f, O = 0.0f;
         if (keff > 0) {
           const float* tab = sm_ptab + (size_t)(g / C) * C * kPartial;
-          float M = -INFINITY;
           for (int r = 0; r < C; ++r) M = fmaxf(M, tab[r * kPartial]);
-          float L = 0.0f, O = 0.0f;
           for (int r = 0; r < C; ++r) {
             const float mr = tab[r * kPartial];
             if (mr == -INFINITY) continue;  // a block that kept no token of this head
@@ -841,10 +924,21 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_ext_kernel(const Deco
           }
           res = O / L;
         }
-        p.out[hq * kDim + e] = res;
+        if constexpr (ATTEND_ONLY) {  // the slice's state (m = -inf, l = 0: it kept no token)
+          float* dst = p.partial + hq * kPartial;
+          dst[4 + e] = O;
+          if (e == 0) {
+            dst[0] = M;
+            dst[1] = L;
+            dst[2] = 0.0f;
+            dst[3] = 0.0f;
+          }
+        } else {
+          p.out[hq * kDim + e] = res;
+        }
       }
     }
-    if (rank == 0)  // slots past k_eff: one row per query head, or one per kv head when shared
+    if (!ATTEND_ONLY && rank == 0)  // slots past k_eff (the sharded step's idx starts at -1): one row per query head, or one per kv head when shared
       for (int i = tid; i < (SHARED ? 1 : G) * p.budget; i += kWorkers) {
         const int g = i / p.budget, r = i - g * p.budget;
         const int64_t row = SHARED ? (int64_t)b * p.Hkv + kvh : (int64_t)b * p.Hq + kvh * G + g;

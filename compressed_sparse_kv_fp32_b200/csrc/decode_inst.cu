@@ -34,7 +34,10 @@ const void* ADAMAS_CAT(decode_fn_g, ADAMAS_DECODE_G)(bool smem_d, int mode) {
       return smem_d ? reinterpret_cast<const void*>(&decode_step_kernel<G, true>)
                     : reinterpret_cast<const void*>(&decode_step_kernel<G, false>);
     case kModeGeneral: return fn_of<kModeGeneral>(smem_d);
-    default: return fn_of<kModeShared>(smem_d);
+    case kModeShared: return fn_of<kModeShared>(smem_d);
+    // the sharded step keeps its distances in the workspace
+    case kModeShardScore: return reinterpret_cast<const void*>(&decode_step_ext_kernel<G, false, kModeShardScore>);
+    default: return reinterpret_cast<const void*>(&decode_step_ext_kernel<G, false, kModeShardAttend>);
   }
 }
 
@@ -46,7 +49,9 @@ cudaError_t ADAMAS_CAT(decode_launch_g, ADAMAS_DECODE_G)(const cudaLaunchConfig_
       return smem_d ? cudaLaunchKernelEx(cfg, decode_step_kernel<G, true>, prm)
                     : cudaLaunchKernelEx(cfg, decode_step_kernel<G, false>, prm);
     case kModeGeneral: return launch_of<kModeGeneral>(cfg, prm, smem_d);
-    default: return launch_of<kModeShared>(cfg, prm, smem_d);
+    case kModeShared: return launch_of<kModeShared>(cfg, prm, smem_d);
+    case kModeShardScore: return cudaLaunchKernelEx(cfg, decode_step_ext_kernel<G, false, kModeShardScore>, prm);
+    default: return cudaLaunchKernelEx(cfg, decode_step_ext_kernel<G, false, kModeShardAttend>, prm);
   }
 }
 

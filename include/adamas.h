@@ -190,12 +190,28 @@ int adamas_score(const void *q, const uint8_t *codes, const int32_t *seq_lens, i
  *     call's contents.  The call clears what must start at zero, but calls that
  *     may overlap on the GPU (different streams, or different threads without
  *     ordering) race on it; serialise them.
- *   - The device error word lives in the shared array and is cleared by the next
- *     call; it cannot be read back through this entry point.
+ *   - The device error word lives in the shared array; every call clears it
+ *     first.  adamas_static_device_error reads the last call's word.
+ *   - The array's address is looked up once per CUDA context (keyed by the
+ *     context's process-unique id) and cached.  cudaDeviceReset destroys the
+ *     context and the array's contents with it; the next call, in the new
+ *     context, looks the address up again.
  */
 int adamas_decode_step_static(const void *q, const uint8_t *codes, const void *K, const void *V,
                               const int32_t *seq_lens, int B, int Hq, int Hkv, int64_t Nmax, int d,
                               int budget, float *out, int32_t *idx, adamas_stream_t stream);
+
+/*
+ * Reads the device error word of the last adamas_decode_step_static call on the
+ * current device (the word lives in the fixed scratch array; see
+ * adamas_get_device_error for its bits).  Synchronises `stream`, so call it on
+ * the stream of the decode calls, after them.  The word stays until the next
+ * static call clears it.
+ * Returns ADAMAS_OK when the word is 0, ADAMAS_ERR_DEVICE when a bit is set
+ * (*error_word holds them), ADAMAS_ERR_INVALID_ARG for a NULL error_word,
+ * ADAMAS_ERR_CUDA when the copy fails.
+ */
+int adamas_static_device_error(uint32_t *error_word, adamas_stream_t stream);
 
 /*
  * Every option of the decode step in one call.  adamas_decode_step and
@@ -278,6 +294,62 @@ int adamas_decode_step_ex(const adamas_decode_args *args, adamas_stream_t stream
  * and not thread-safe: for the tests of the timeout path only.
  */
 void adamas_debug_withhold_stage(int stage);
+
+/*
+ * Sequence-sharded decode step, for contexts longer than one GPU holds (the 2M-token
+ * context blog, intelliparadigm.com/.../2174157, §5.1: two million tokens need
+ * several GPUs or CPU offloading; the AMD Zebra-HyLo article,
+ * yeyulingfeng.com/a/1106654.html, reports 2M-token contexts).  Each of `world`
+ * GPUs holds one contiguous slice of every sequence (rank r the r-th slice, in
+ * sequence order) in its own codes/K/V arrays, [B][Hkv][Nmax][...] as above with
+ * seq_lens[b] the slice's length.  One step, on every rank:
+ *   1. adamas_shard_score: scores the slice; writes the slice's distance
+ *      histograms to `hist` [B][Hq][ADAMAS_HIST_STRIDE] uint32 (bins 0..384).
+ *   2. all-gather of `hist` in rank order -> hist_all [world][B][Hq][ADAMAS_HIST_STRIDE].
+ *   3. adamas_shard_attend: from hist_all, the threshold and rank bases of the
+ *      whole sequence (k_eff = min(budget, total length)); the slice's kept tokens
+ *      get their slots, idx [B][Hq][budget] holds their indices in the whole
+ *      sequence (every other slot -1), and `partial` [B][Hq][ADAMAS_PARTIAL_FLOATS]
+ *      fp32 receives the slice's softmax state over them.
+ *   4. all-gather of `partial` -> [world][B][Hq][ADAMAS_PARTIAL_FLOATS], and an
+ *      all-reduce (max) of idx.
+ *   5. adamas_merge_partials -> out [B][Hq][128].
+ * The result is the step of adamas_decode_step on the whole sequence: the same
+ * idx, and out within the float tolerance of the single-GPU step.  Per head and
+ * rank the messages are 388 * 4 B (histograms) and 132 * 4 B (state) plus the idx
+ * row.  Per-head selection only (no forced rows, paged cache, group-shared policy
+ * or append); global indices are int32, so a sequence holds at most 2^31 - 1 tokens.
+ *
+ * The workspace (adamas_shard_workspace_bytes, initialised once with
+ * adamas_workspace_init) carries the slice's distances and per-block histograms
+ * from step 1 to step 3: use the same workspace, stream and shape for both.
+ * `hist` and idx are overwritten (zeroed / set to -1) by the calls themselves.
+ * A partial state is (m, l, 0, 0, o[128]): m the largest score of the slice's kept
+ * tokens, in log2 units (q.k / sqrt(128) * log2 e), l = sum 2^(s - m) and
+ * o = sum 2^(s - m) v over them; m = -inf and l = 0 when the slice kept none.
+ * Errors as for adamas_decode_step; the device error word is the workspace's.
+ */
+#define ADAMAS_HIST_STRIDE 388
+#define ADAMAS_PARTIAL_FLOATS 132
+
+size_t adamas_shard_workspace_bytes(int B, int Hq, int Hkv, int64_t Nmax, int d, int budget);
+
+int adamas_shard_score(const void *q, const uint8_t *codes, const int32_t *seq_lens, int B, int Hq, int Hkv,
+                       int64_t Nmax, int d, int budget, uint32_t *hist, void *workspace, size_t workspace_bytes,
+                       adamas_stream_t stream);
+
+/* world >= 1 ranks, 0 <= rank < world; hist_all as gathered in step 2. */
+int adamas_shard_attend(const void *q, const void *K, const void *V, const int32_t *seq_lens, int B, int Hq, int Hkv,
+                        int64_t Nmax, int d, int budget, const uint32_t *hist_all, int world, int rank,
+                        float *partial, int32_t *idx, void *workspace, size_t workspace_bytes,
+                        adamas_stream_t stream);
+
+/*
+ * out[b][h][e] = sum_r 2^(m_r - M) o_r[e] / sum_r 2^(m_r - M) l_r over the n states
+ * partials [n][B][Hq][ADAMAS_PARTIAL_FLOATS] (M = max_r m_r; states with m_r = -inf
+ * are skipped; 0 when every state is empty).  16-byte aligned fp32 arrays.
+ */
+int adamas_merge_partials(const float *partials, int n, int B, int Hq, float *out, adamas_stream_t stream);
 
 /*
  * Synchronise `stream`, then copy the workspace's device error word into

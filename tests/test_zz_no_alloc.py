@@ -38,7 +38,9 @@ def _static_call(lib, q, codes, K, V, lens, budget, out, idx):
 
 
 @pytest.mark.parametrize("wid,kw,budget", [(2, dict(Hq=8, Hkv=8, Nmax=20000), 256),
-                                           (4, dict(B=3, Nmax=5000, len_range=(100, 5000)), 64)])
+                                           (4, dict(B=3, Nmax=5000, len_range=(100, 5000)), 64),
+                                           # G = 8 over 200K tokens: the distances spill into the scratch
+                                           (5, dict(B=1, Hq=8, Hkv=1, Nmax=200000, len_range=None), 512)])
 def test_matches_workspace_entry_point_twice(wid, kw, budget):
     lib = adamas.load()
     w = synth.WORKLOADS[wid].scaled(**kw)
@@ -55,6 +57,27 @@ def test_matches_workspace_entry_point_twice(wid, kw, budget):
         torch.cuda.synchronize()
         assert np.array_equal(idx.cpu().numpy(), ref_idx.cpu().numpy())
         assert_close_out(out.cpu().numpy(), ref_out.cpu().numpy())
+        word = ctypes.c_uint32(7)
+        assert lib.adamas_static_device_error(ctypes.byref(word), torch.cuda.current_stream().cuda_stream) == 0
+        assert word.value == 0
+
+
+def test_device_errors_of_the_static_path_can_be_read_back():
+    lib = adamas.load()
+    w = synth.WORKLOADS[2].scaled(Hq=2, Hkv=2, Nmax=3000)
+    inp, K, V, codes = _inputs(w)
+    q = dev_bf16(inp["q"])
+    out = torch.empty((1, 2, 128), dtype=torch.float32, device="cuda")
+    idx = torch.empty((1, 2, 64), dtype=torch.int32, device="cuda")
+    st = torch.cuda.current_stream().cuda_stream
+    word = ctypes.c_uint32(0)
+    bad = dev(np.array([w.Nmax + 5], np.int32))      # beyond the cache: clamped and flagged
+    assert _static_call(lib, q, codes, K, V, bad, 64, out, idx) == 0
+    rc = lib.adamas_static_device_error(ctypes.byref(word), st)
+    assert rc == -5 and word.value & adamas.DEVERR_SEQLEN  # ADAMAS_ERR_DEVICE
+    good = dev(np.array([w.Nmax], np.int32))          # the next call clears the word
+    assert _static_call(lib, q, codes, K, V, good, 64, out, idx) == 0
+    assert lib.adamas_static_device_error(ctypes.byref(word), st) == 0 and word.value == 0
 
 
 def test_sizes_beyond_the_fixed_scratch_are_rejected():
