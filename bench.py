@@ -10,11 +10,18 @@ buffers rotate so that the working set is far larger than L2.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
                     [--workload NAME] [--budget K] [--policy per_head|group_shared]
+                    [--slices S]
 
 Prints one JSON line.  --impl reference times the CPU oracle on a bounded sample
 of the same workload.  Under torchrun every rank runs its own independent copy of
 the workload (weak scaling, no collective on the data path); the time is the max
 over ranks.
+
+--slices S times the sequence-sharded step instead: every sequence split into S
+contiguous slices.  Under torchrun S must equal the number of ranks (one slice per
+GPU, histograms and softmax states exchanged over NCCL); on one GPU the S slices
+are emulated one after the other (their kernels run in turn, the exchanges are
+local stacks), so the time is the sum of the S slices' work.
 """
 from __future__ import annotations
 
@@ -59,6 +66,7 @@ def parse():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(DEFAULT_BUDGET))
     ap.add_argument("--budget", type=int, default=None)
     ap.add_argument("--policy", default="per_head", choices=["per_head", "group_shared"])
+    ap.add_argument("--slices", type=int, default=0, help="time the sequence-sharded step over S slices")
     a = ap.parse_args()
     if a.budget is None:
         a.budget = DEFAULT_BUDGET[a.workload]
@@ -447,6 +455,104 @@ def run_gpu(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def run_sharded(args, rank, world):
+    """The sequence-sharded step (see the module docstring for --slices)."""
+    import torch
+
+    from compressed_sparse_kv_fp32_b200 import adamas, sharded
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = workload_of(args.workload)
+    B, Hq, Hkv, d, budget = w.B, w.Hq, w.Hkv, w.d, args.budget
+    S = args.slices
+    if world > 1 and S != world:
+        raise SystemExit("--slices must equal the number of ranks under torchrun")
+    mine = [rank] if world > 1 else list(range(S))
+    lens_np = synth.seq_lens(w)
+    bounds = [[sharded.slice_bounds(int(n), S, r) for n in lens_np] for r in range(S)]
+
+    def to_dev(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(torch.bfloat16)
+
+    slices = {}
+    for r in mine:
+        ln = np.array([e - a for a, e in bounds[r]], np.int32)
+        nmax = max(1, int(ln.max()))
+        K = torch.zeros((B, Hkv, nmax, d), dtype=torch.bfloat16, device=dev)
+        V = torch.zeros_like(K)
+        for b in range(B):
+            a, e = bounds[r][b]
+            for h in range(Hkv):
+                k, v = synth.head_kv(w, b, h)
+                K[b, h, :e - a] = to_dev(k[a:e])
+                V[b, h, :e - a] = to_dev(v[a:e])
+        codes = torch.empty((B, Hkv, nmax, 32), dtype=torch.uint8, device=dev)
+        adamas.encode_keys(K, codes)
+        slices[r] = dict(K=K, V=V, codes=codes, lens=torch.from_numpy(ln).to(dev),
+                         ops=sharded.CudaShardOps(B, Hq, Hkv, nmax, budget, device=dev))
+    q = to_dev(synth.query(w, 1))
+    torch.cuda.synchronize()
+
+    if world > 1:
+        ex = sharded.TorchExchange()
+        sl = slices[rank]
+
+        def step():
+            return sharded.decode_step_sharded(q, sl["codes"], sl["K"], sl["V"], sl["lens"], budget, sl["ops"], ex)
+    else:
+        def step():
+            hist_all = torch.stack([slices[r]["ops"].score(q, slices[r]["codes"], slices[r]["lens"], budget)
+                                    for r in mine], 0)
+            st = [slices[r]["ops"].attend(q, slices[r]["K"], slices[r]["V"], slices[r]["lens"], budget, hist_all, r)
+                  for r in mine]
+            idx = st[0][1]
+            for _, i in st[1:]:
+                idx = torch.maximum(idx, i)
+            return slices[mine[0]]["ops"].merge(torch.stack([p for p, _ in st], 0)), idx
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(args.steps):
+        step()
+    t1.record()
+    torch.cuda.synchronize()
+    (elapsed_ms,) = max_over_ranks([t0.elapsed_time(t1)], dev)
+    for r in mine:
+        if slices[r]["ops"].workspace.device_error() != 0:
+            raise RuntimeError("device error word set during the sharded bench")
+    if rank != 0:
+        return
+    ms = elapsed_ms / args.steps
+    step_bytes = accounting.decode_step_bytes(lens_np, Hq, Hkv, budget, d)
+    # the sharded step also writes and reads back every distance (2 B per token and query head)
+    spill = 2 * 2 * int(lens_np.sum()) * Hq
+    line = {
+        "metric": f"sharded decode steps/s, {w.name}, budget {budget}, {S} slices"
+                  + (" emulated on one GPU" if world == 1 else " on as many GPUs"),
+        "value": 1e3 / ms, "unit": "decode steps/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+        "dtype": "u8/fp32", "data": "synthetic",
+        "config": dict(config_block(w, args), slices=S,
+                       workload=f"{w.name}: batch {B}, {Hq} query heads over {Hkv} kv heads, context {w.Nmax}, "
+                                f"budget {budget}, sequences split into {S} contiguous slices, no append",
+                       l2=f"one buffer per slice, codes of all slices {B * Hkv * w.Nmax * 32 / 2**30:.2f} GiB",
+                       parallelism=f"sequence-sharded over {S} slices"),
+        "algorithmic_bytes_per_step": step_bytes["total"] + spill,
+        "achieved_gbs": (step_bytes["total"] + spill) / (ms / 1e3) / 1e9,
+        "exchange_bytes_per_rank": {"histograms": B * Hq * adamas.HIST_STRIDE * 4,
+                                    "states": B * Hq * adamas.PARTIAL_FLOATS * 4, "idx": B * Hq * budget * 4},
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -463,7 +569,7 @@ def main():
         torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     try:
-        run_gpu(args, rank, world)
+        (run_sharded if args.slices > 0 else run_gpu)(args, rank, world)
     finally:
         if world > 1:
             import torch.distributed as dist

@@ -28,16 +28,19 @@
 //            kept; of the ties D == T this block keeps its first k_eff - base(T)
 //            in index order, so ties go to the lowest indices.  A token's output
 //            slot is its rank base + its rank by index among the block's tokens
-//            of equal distance.  One pass over the block's distances puts every
-//            token with D <= T (typically a few hundred) into its distance group
-//            (atomic cursors; each thread walks its own run of positions, lanes
-//            rotated so that a warp's loads spread over the banks), and each
-//            token is then ranked inside its group.  When groups are large (heavy
-//            ties) two scans take over: per-warp counts, then an in-order emit
-//            with a warp match over 32-entry chunks for the D < T tokens.  Either
-//            way the kept tokens end up in slot order, so both give the same bits.
-//            The kept K/V rows are prefetched into L2, gathered into registers
-//            (each half-warp keeps four K and four V rows in flight) and folded
+//            of equal distance.  One pass over the block's distances lists every
+//            token with D <= T (typically a few hundred) in index order (each
+//            thread marks its own run of positions, lanes rotated so that a warp's
+//            loads spread over the banks; one block scan of the counts gives each
+//            thread its place in the list); a token's rank among the block's tokens
+//            of its distance is then the number of listed tokens of that distance
+//            before it (a warp match, per-warp counts, counts carried between
+//            rounds of 512 entries).  When more than 4096 tokens have D <= T (heavy
+//            ties) two scans take over: per-warp counts, then an in-order emit with
+//            a warp match over 32-entry chunks for the D < T tokens.  Either way
+//            the kept tokens end up in slot order, so both give the same bits.
+//            The kept K/V rows are gathered into registers (each half-warp keeps
+//            four K and four V rows in flight) and folded
 //            into an online-softmax state per half-warp; the states become one
 //            partial (m, l, o) per query head and block, which goes to the block
 //            that owns the head's merge.
@@ -73,7 +76,6 @@ constexpr int kHistStride = 388;                      // >= kBins, multiple of 4
 constexpr int kPartial = 132;                         // m, l, pad, pad, o[128]
 constexpr int kListCap = 4096;                        // D < T tokens listed per round / grouped tokens D <= T
 constexpr int kKeptCap = 4096;                        // kept tokens per gather window
-constexpr int kGroupMax = 512;                        // largest equal-distance group ranked pairwise
 constexpr int kGatherRows = 4;                        // K/V rows in flight per half-warp
 constexpr int kScanBatch = 4;                         // 32-group iterations of a distance scan loaded together
 constexpr int kGatherBatch = 2 * kWorkerWarps * kGatherRows;  // rows per gather batch of the block

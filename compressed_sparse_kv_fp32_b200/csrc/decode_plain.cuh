@@ -21,7 +21,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const DecodePa
   __shared__ int sm_wmax[kWorkerWarps];
   __shared__ uint32_t sm_acode[kCodeWords];  // the appended key's code
   __shared__ long long sm_tmp[kWorkerWarps];
-  __shared__ uint32_t sm_sink[32];  // per-lane target of the unused atomics of a batch
 
   cg::cluster_group cluster = cg::this_cluster();
   const int C = p.cluster;
@@ -287,20 +286,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const DecodePa
       const int n_kept = n_lt + min(tie_quota, n_eq);   // kept tokens, in slot order at [0, n_kept)
       const uint4 qraw = *reinterpret_cast<const uint4*>(p.q + hq * kDim + 8 * hl);
 
-      // largest group of equal distances <= T, and whether the candidate list serves
-      {
-        const int v = (tid <= (int)T) ? (int)hist_g[tid] : 0;
-        const int m = __reduce_max_sync(0xffffffffu, v);
-        if (lane == 0) sm_wmax[warp] = m;
-      }
-      for (int i = tid; i < kHistStride; i += kWorkers) sm_carry[i] = 0u;
-      worker_sync();
-      int gmax = 0;
-#pragma unroll
-      for (int w = 0; w < kWorkerWarps; ++w) gmax = max(gmax, sm_wmax[w]);
-      // grouped path: every token with D <= T grouped by distance and ranked inside
-      // its group; else the two scans
-      bool grouped = n_lt + n_eq <= kListCap && n_kept <= kKeptCap && gmax <= kGroupMax;
+      // The compact path: every token with D <= T (typically a few hundred) is listed
+      // in index order, then ranked among the listed tokens of its distance; else the
+      // two scans.
+      bool compact = n_lt + n_eq <= kListCap && n_kept <= kKeptCap;
 
       float qf[8];
       float m_run = -INFINITY, l_run = 0.0f, o[8];
@@ -320,84 +309,95 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const DecodePa
         }
       };
 
-      if (grouped) {
-        // ---- every token with D <= T to its group (group d at [lpre[d], lpre[d] + hist[d])):
-        // each thread takes a run of 8-position groups, eight at a time (lanes start
-        // at different points of the eight so that a warp's loads spread over the
-        // banks), and places its candidates four at a time so that their atomic
-        // cursor updates are in flight together
+      if (compact) {
+        // ---- list: rounds over consecutive spans of at most kWorkers * 8 groups of 8
+        // positions; in a round each thread takes a run of at most eight groups (lanes
+        // start at different points of the eight so that a warp's loads spread over the
+        // banks) and marks D <= T, and after one block scan of the counts writes its
+        // tokens -- (D << 23 | offset) -- from its offset on, so the list is in index
+        // order.
         const uint32_t t1x2 = (T + 1) | (T + 1) << 16;
-        const int chunk = (ngrp + kWorkers - 1) / kWorkers;
         const int rot = lane & 7;
-        for (int k0 = 0; k0 < chunk; k0 += 8) {
-          unsigned long long cm = 0ull;  // bit 8j + e: position (tid * chunk + k0 + j) * 8 + e
+        for (int i = tid; i < kWorkerWarps * kHistStride; i += kWorkers) sm_cnt[i] = 0u;
+        for (int i = tid; i < kHistStride; i += kWorkers) sm_carry[i] = 0u;
+        int listed = 0;  // tokens listed by earlier rounds
+        for (int r0 = 0; r0 < ngrp; r0 += kWorkers * 8) {
+          const int span = min(kWorkers * 8, ngrp - r0);
+          const int cnt = (span + kWorkers - 1) / kWorkers;
+          const int g0 = r0 + tid * cnt;
+          unsigned long long cm = 0ull;  // bit 8j + e: position (g0 + j) * 8 + e
 #pragma unroll
           for (int h = 0; h < 8; h += 2) {
             uint4 v[2];
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
-              const int j = (h + u + rot) & 7, grp = tid * chunk + k0 + j;
-              v[u] = (k0 + j < chunk && grp < ngrp) ? load_dist8<SMEM_D>(drow, grp)
-                                                    : make_uint4(~0u, ~0u, ~0u, ~0u);
+              const int j = (h + u + rot) & 7, grp = g0 + j;
+              v[u] = (j < cnt && grp < r0 + span) ? load_dist8<SMEM_D>(drow, grp)
+                                                  : make_uint4(~0u, ~0u, ~0u, ~0u);
             }
 #pragma unroll
             for (int u = 0; u < 2; ++u) cm |= (unsigned long long)le_bits(v[u], t1x2) << (8 * ((h + u + rot) & 7));
           }
-          while (cm != 0ull) {
-            uint32_t tp[4], dd[4], cc[4];
-            bool ok[4];
+          const int mine = __popcll((long long)cm);
+          const uint32_t before = worker_exclusive_scan32((uint32_t)mine, reinterpret_cast<uint32_t*>(sm_tmp));
+          if (tid == kWorkers - 1) sm_wmax[0] = (int)before + mine;
+          int at = listed + (int)before;
+          for (; cm != 0ull; cm &= cm - 1ull, ++at) {
+            const int bit = __ffsll((long long)cm) - 1;
+            const uint32_t pos = (uint32_t)((g0 + (bit >> 3)) * 8 + (bit & 7));
+            const uint32_t dd = load_dist1<SMEM_D>(drow, (int)pos);
+            if (at < kListCap) sm_list[at] = (int32_t)(dd << 23 | pos);
+          }
+          worker_sync();  // the round's total is visible
+          listed += sm_wmax[0];
+          worker_sync();  // every thread has read it before the next round overwrites it
+        }
+        if (listed != n_lt + n_eq) {  // never with consistent histograms
+          if (tid == 0) atomicOr(p.err, kErrInternal);
+          listed = min(listed, kListCap);
+        }
+        // ---- slots: a token's rank among the block's tokens of its distance is the
+        // number of listed tokens of that distance before it (the list is in index
+        // order): per round of kWorkers entries, a warp match gives the rank inside the
+        // warp, per-warp counts give the warps before, carried counts the rounds before
+        for (int r0 = 0; r0 < listed; r0 += kWorkers) {
+          const int i = r0 + tid;
+          const bool valid = i < listed;
+          const uint32_t ent = valid ? lds32(smem_addr(sm_list + i)) : 0u;
+          const uint32_t d = ent >> 23, tpos = ent & kPosMask;
+          const uint32_t vm = __ballot_sync(0xffffffffu, valid);
+          uint32_t peers = 0u;
+          if (valid) {
+            peers = __match_any_sync(vm, d);
+            if ((peers & lt) == 0u) sm_cnt[warp * kHistStride + d] = (uint32_t)__popc(peers);
+          }
+          worker_sync();
+          if (valid) {
+            const uint32_t ca = smem_addr(sm_cnt + d);
+            uint32_t before = lds32(smem_addr(sm_carry + d)) + (uint32_t)__popc(peers & lt);
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              ok[u] = cm != 0ull;
-              const int bit = ok[u] ? __ffsll((long long)cm) - 1 : 0;
-              cm &= cm - 1ull;
-              tp[u] = ok[u] ? (uint32_t)((tid * chunk + k0 + (bit >> 3)) * 8 + (bit & 7)) : 0u;
-            }
-#pragma unroll
-            for (int u = 0; u < 4; ++u) dd[u] = load_dist1<SMEM_D>(drow, (int)tp[u]);
-#pragma unroll
-            for (int u = 0; u < 4; ++u) cc[u] = atomicAdd(ok[u] ? &sm_carry[dd[u]] : &sm_sink[lane], 1u);
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              if (!ok[u] || cc[u] >= hist_g[dd[u]]) continue;  // the latter never with consistent histograms
-              sm_list[lpre_g[dd[u]] + cc[u]] = (int32_t)(dd[u] << 23 | tp[u]);
-              const int64_t row = kv_base + t0 + tp[u];  // the row is very likely kept: on its way into L2
-              prefetch_l2(p.K + row * kDim);
-              prefetch_l2(p.K + row * kDim + 64);
-              prefetch_l2(p.V + row * kDim);
-              prefetch_l2(p.V + row * kDim + 64);
+            for (int w = 0; w < kWorkerWarps - 1; ++w)
+              if (w < warp) before += lds32(ca + w * kHistStride * 4);
+            const uint32_t slot = rank_g[d] + before;
+            const uint32_t kp = lpre_g[d] + before;
+            if (slot < (uint32_t)keff && kp < (uint32_t)n_kept) {
+              idx_h[slot] = (int32_t)(t0 + tpos);
+              sm_kept[kp] = (int32_t)tpos;
             }
           }
-        }
-        worker_sync();
-        // every group must be complete (each token with D <= T placed once), else the scans decide
-        if (tid == 0) sm_wmax[0] = 0;
-        worker_sync();
-        if (tid <= (int)T && sm_carry[tid] != hist_g[tid]) sm_wmax[0] = 1;
-        worker_sync();
-        grouped = sm_wmax[0] == 0;
-        worker_sync();
-      }
-      if (grouped) {
-        // ---- rank inside the group by index: slot, and the kept position lpre[d] + rank
-        const int nf = n_lt + n_eq;
-        for (int i = tid; i < nf; i += kWorkers) {
-          const uint32_t e = lds32(smem_addr(sm_list + i));
-          const uint32_t d = e >> 23, tpos = e & kPosMask;
-          const int gb = (int)lpre_g[d], gn = (int)hist_g[d];
-          const int32_t* grp_list = sm_list + gb;  // plain loads: the compiler keeps several in flight
-          int r = 0, q = 0;
-          for (; q + 4 <= gn; q += 4)
-            r += (((uint32_t)grp_list[q] & kPosMask) < tpos) + (((uint32_t)grp_list[q + 1] & kPosMask) < tpos) +
-                 (((uint32_t)grp_list[q + 2] & kPosMask) < tpos) + (((uint32_t)grp_list[q + 3] & kPosMask) < tpos);
-          for (; q < gn; ++q) r += ((uint32_t)grp_list[q] & kPosMask) < tpos;
-          const int slot = (int)rank_g[d] + r;
-          if (slot < keff) {
-            idx_h[slot] = (int32_t)(t0 + tpos);
-            sm_kept[gb + r] = (int32_t)tpos;
+          if (r0 + kWorkers < listed) {  // counts carried to the next round
+            worker_sync();
+            for (int dd = tid; dd < kBins; dd += kWorkers) {
+              uint32_t c = 0u;
+              for (int w = 0; w < kWorkerWarps; ++w) {
+                c += sm_cnt[w * kHistStride + dd];
+                sm_cnt[w * kHistStride + dd] = 0u;
+              }
+              sm_carry[dd] += c;
+            }
           }
+          worker_sync();
         }
-        worker_sync();
         qf[0] = bf16_lo(qraw.x) * kScoreScale; qf[1] = bf16_hi(qraw.x) * kScoreScale;
         qf[2] = bf16_lo(qraw.y) * kScoreScale; qf[3] = bf16_hi(qraw.y) * kScoreScale;
         qf[4] = bf16_lo(qraw.z) * kScoreScale; qf[5] = bf16_hi(qraw.z) * kScoreScale;
@@ -405,7 +405,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const DecodePa
         gather(n_kept, false);
         worker_sync();
       }
-      if (!grouped) {
+      if (!compact) {
         // ---- count pass: candidates per warp
         const uint32_t tx2 = T | T << 16, t1x2 = (T + 1) | (T + 1) << 16;
         int c_lt = 0, c_eq = 0;
