@@ -525,6 +525,24 @@ def run_sharded(args, rank, world):
     t1.record()
     torch.cuda.synchronize()
     (elapsed_ms,) = max_over_ranks([t0.elapsed_time(t1)], dev)
+    # per slice: its two kernels alone (score, then attend with the gathered
+    # histograms), the time one GPU of a real sharded step spends in kernels
+    per_slice = None
+    if world == 1:
+        hist_all = torch.stack([slices[r]["ops"].score(q, slices[r]["codes"], slices[r]["lens"], budget)
+                                for r in mine], 0)
+        per_slice = []
+        for r in mine:
+            sl = slices[r]
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+            reps = max(1, args.steps // 4)
+            ev[0].record()
+            for _ in range(reps):
+                sl["ops"].score(q, sl["codes"], sl["lens"], budget)
+                sl["ops"].attend(q, sl["K"], sl["V"], sl["lens"], budget, hist_all, r)
+            ev[1].record()
+            torch.cuda.synchronize()
+            per_slice.append(ev[0].elapsed_time(ev[1]) / reps * 1e3)
     for r in mine:
         if slices[r]["ops"].workspace.device_error() != 0:
             raise RuntimeError("device error word set during the sharded bench")
@@ -547,6 +565,7 @@ def run_sharded(args, rank, world):
                        parallelism=f"sequence-sharded over {S} slices"),
         "algorithmic_bytes_per_step": step_bytes["total"] + spill,
         "achieved_gbs": (step_bytes["total"] + spill) / (ms / 1e3) / 1e9,
+        "per_slice_kernel_us": per_slice,
         "exchange_bytes_per_rank": {"histograms": B * Hq * adamas.HIST_STRIDE * 4,
                                     "states": B * Hq * adamas.PARTIAL_FLOATS * 4, "idx": B * Hq * budget * 4},
     }

@@ -184,8 +184,6 @@ int adamas_score(const void *q, const uint8_t *codes, const int32_t *seq_lens, i
  *   - Sizes whose workspace (adamas_workspace_bytes) exceeds 4 MiB are rejected
  *     with ADAMAS_ERR_WORKSPACE before anything is enqueued; use
  *     adamas_decode_step for those.
- *   - The first call on each device looks up the array's device address (a
- *     one-time set-up); make that first call before any stream capture.
  *   - Every call on a device shares the one array, and it keeps the previous
  *     call's contents.  The call clears what must start at zero, but calls that
  *     may overlap on the GPU (different streams, or different threads without
