@@ -10,12 +10,15 @@ buffers rotate so that the working set is far larger than L2.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
                     [--workload NAME] [--budget K] [--policy per_head|group_shared]
-                    [--slices S]
+                    [--slices S] [--page-size P]
 
 Prints one JSON line.  --impl reference times the CPU oracle on a bounded sample
 of the same workload.  Under torchrun every rank runs its own independent copy of
 the workload (weak scaling, no collective on the data path); the time is the max
 over ranks.
+
+--page-size P keeps every layer's cache in pages of P tokens, [n_pages][Hkv][P][...],
+placed in a shuffled order and read through a block table (the step with options).
 
 --slices S times the sequence-sharded step instead: every sequence split into S
 contiguous slices.  Under torchrun S must equal the number of ranks (one slice per
@@ -67,6 +70,8 @@ def parse():
     ap.add_argument("--budget", type=int, default=None)
     ap.add_argument("--policy", default="per_head", choices=["per_head", "group_shared"])
     ap.add_argument("--slices", type=int, default=0, help="time the sequence-sharded step over S slices")
+    ap.add_argument("--page-size", type=int, default=0,
+                    help="read the cache through a block table of pages of this many tokens (shuffled pages)")
     a = ap.parse_args()
     if a.budget is None:
         a.budget = DEFAULT_BUDGET[a.workload]
@@ -78,10 +83,11 @@ def workload_of(name):
 
 
 def metric_of(args, w):
-    if args.workload == DEFAULT_WORKLOAD and args.budget == 1024 and args.policy == "per_head":
+    if args.workload == DEFAULT_WORKLOAD and args.budget == 1024 and args.policy == "per_head" and not args.page_size:
         return METRIC
     return (f"decode steps/s and achieved HBM GB/s (% of B200 peak): {w.name}, context {w.Nmax}, "
-            f"budget {args.budget}, {args.policy.replace('_', '-')} selection")
+            f"budget {args.budget}, {args.policy.replace('_', '-')} selection"
+            + (f", paged cache ({args.page_size}-token pages)" if args.page_size else ""))
 
 
 def source_hash() -> str:
@@ -274,9 +280,26 @@ def run_gpu(args, rank, world):
                 Ks[l][b, h].copy_(kd)
                 Vs[l][b, h].copy_(vd)
             new_k[b, h], new_v[b, h] = k[lens_np[b] - 1], v[lens_np[b] - 1]
+    P = args.page_size
+    table = None
+    if P > 0:  # pages of P tokens in a shuffled physical order, read through a block table
+        max_pages = (N + P - 1) // P
+        n_pages = B * max_pages
+        perm = torch.from_numpy(np.random.default_rng(7).permutation(n_pages)).to(dev)
+        table = perm.to(torch.int32).view(B, max_pages).contiguous()
+        for l in range(n_layers):
+            for X in (Ks, Vs):
+                pad = torch.zeros((B, Hkv, max_pages * P, d), dtype=torch.bfloat16, device=dev)
+                pad[:, :, :N] = X[l]
+                logical = pad.view(B, Hkv, max_pages, P, d).permute(0, 2, 1, 3, 4).reshape(n_pages, Hkv, P, d)
+                phys = torch.empty((n_pages, Hkv, P, d), dtype=torch.bfloat16, device=dev)
+                phys[perm] = logical
+                X[l] = phys
+                del pad, logical
+        N = max_pages * P
     layers = []
     for l in range(n_layers):
-        codes = torch.empty((B, Hkv, N, 32), dtype=torch.uint8, device=dev)
+        codes = torch.empty(tuple(Ks[l].shape[:3]) + (32,), dtype=torch.uint8, device=dev)
         adamas.encode_keys(Ks[l], codes)
         q = to_dev(synth.query(w, l + 1))
         out = torch.empty((B, Hq, d), dtype=torch.float32, device=dev)
@@ -309,7 +332,9 @@ def run_gpu(args, rank, world):
         argss.append(adamas.DecodeArgs(
             L["q"].data_ptr(), L["codes"].data_ptr(), L["K"].data_ptr(), L["V"].data_ptr(), lens.data_ptr(),
             B, Hq, Hkv, N, d, budget, L["out"].data_ptr(), L["idx"].data_ptr(), L["ws"].buffer.data_ptr(),
-            L["ws"].nbytes, pos.data_ptr(), None, None, None, 0, 0, 0, 0, 0,
+            L["ws"].nbytes, pos.data_ptr(), None, None,
+            None if table is None else table.data_ptr(), 0 if table is None else table.numel(),
+            P if table is not None else 0, table.shape[1] if table is not None else 0, 0, 0,
             adamas.SELECT_GROUP_SHARED if shared else adamas.SELECT_PER_HEAD))
     refs = [ctypes.byref(a) for a in argss]
     f_step = lib.adamas_decode_step_ex
@@ -391,7 +416,7 @@ def run_gpu(args, rank, world):
         L = layers[i % n_layers]
         in_dev.copy_(in_pin, non_blocking=True)
         adamas.decode(q_dev, L["codes"], L["K"], L["V"], lens, budget, L["ws"], append_pos=pos, k_new=krow_dev,
-                      v_new=vrow_dev, policy=policy, out=out_dev, idx=idx_dev)
+                      v_new=vrow_dev, block_table=table, policy=policy, out=out_dev, idx=idx_dev)
         res_pin.copy_(res_dev, non_blocking=True)
         torch.cuda.current_stream().synchronize()
 
@@ -420,17 +445,19 @@ def run_gpu(args, rank, world):
     launch_bytes = step_bytes["total"] + enc_bytes   # the launch also encodes the appended keys
     achieved_dec = launch_bytes / (dec_ms / 1e3) / 1e9
     achieved_step = launch_bytes / (ms_per_step / 1e3) / 1e9
-    headline = args.workload == DEFAULT_WORKLOAD and budget == 1024 and not shared
+    headline = args.workload == DEFAULT_WORKLOAD and budget == 1024 and not shared and not P
     traffic = profiled_traffic("decode_step_kernel_mha32_128k") if headline else None
     enc_all = B * Hkv * N * accounting.encode_bytes_per_vector(d)
     line = {
         "metric": metric_of(args, w), "value": value, "unit": UNIT, "n_gpus": world, "steps": K_steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "u8/fp32", "data": "synthetic",
-        "config": config_block(w, args, n_layers),
+        "config": dict(config_block(w, args, n_layers),
+                       **({"page_size": P, "cache": f"{B * ((w.Nmax + P - 1) // P)} pages of {P} tokens in shuffled "
+                           "order, read through a block table"} if P > 0 else {})),
         "achieved_hbm_gbs": achieved_step, "pct_of_peak_hbm": 100.0 * achieved_step / peak,
         "peak_hbm_gbs": peak, "peak_kind": peak_kind,
-        "roofline": {"bound": "hbm", "kernel": "decode_step_kernel" if not shared else "decode_step_ext_kernel",
+        "roofline": {"bound": "hbm", "kernel": "decode_step_kernel" if not (shared or P) else "decode_step_ext_kernel",
                      "achieved": achieved_dec, "peak": peak,
                      "unit": "GB/s", "frac": achieved_dec / peak, "traffic": traffic,
                      "algorithmic_bytes_per_launch": launch_bytes, "avg_launch_us": dec_ms * 1e3,

@@ -365,16 +365,24 @@ __device__ __forceinline__ void gather_fold(int rb, int n, int hw, const float (
 
 // Cache row of token t of (b, kv head): [B][Hkv][Nmax] when contiguous; through
 // the block table otherwise, pages laid out [page][Hkv][page_size].  An entry
-// outside [0, n_pages) is flagged and read as page 0 (accesses stay in bounds).
-__device__ __forceinline__ int64_t cache_row(const DecodeParams& p, int b, int kvh, int64_t t) {
+// outside [0, n_pages) reads page 0 (accesses stay in bounds) and sets `bad`; the
+// caller flags it.  No branch depends on the table entry, so a warp does not stall
+// on the table read until it uses the row.
+__device__ __forceinline__ int64_t cache_row(const DecodeParams& p, int b, int kvh, int64_t t, bool& bad) {
   if (p.table == nullptr) return ((int64_t)b * p.Hkv + kvh) * p.Nmax + t;
-  const int lp = (int)(t / p.page_size), off = (int)(t - (int64_t)lp * p.page_size);
-  int64_t page = p.table[(int64_t)b * p.max_pages + lp];
-  if (page < 0 || page >= p.n_pages) {
-    atomicOr(p.err, kErrTable);
-    page = 0;
-  }
-  return (page * p.Hkv + kvh) * p.page_size + off;
+  const int lp = (int)((uint32_t)t / (uint32_t)p.page_size);  // t < 2^31
+  const int off = (int)t - lp * p.page_size;
+  const int64_t page = p.table[(int64_t)b * p.max_pages + lp];
+  const bool ok = page >= 0 && page < p.n_pages;
+  bad |= !ok;
+  return ((ok ? page : 0) * p.Hkv + kvh) * p.page_size + off;
+}
+
+__device__ __forceinline__ int64_t cache_row(const DecodeParams& p, int b, int kvh, int64_t t) {
+  bool bad = false;
+  const int64_t r = cache_row(p, b, kvh, t, bad);
+  if (bad) atomicOr(p.err, kErrTable);
+  return r;
 }
 
 }  // namespace adamas

@@ -184,9 +184,22 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_ext_kernel(const Deco
     // Stage i holds the code rows of tokens t0 + [i * kStageRows, +rows): one bulk copy
     // in a contiguous cache; in a paged cache lane 0 waits for the stage to be free and
     // arms its barrier with the stage's bytes, and the lanes copy one page piece each.
+    // The lane's first kLookAhead page pieces of a stage are looked up in the block
+    // table before the wait for the stage's buffer, so the table reads overlap it
+    // (a bad entry is flagged once, after the stream).
+    constexpr int kLookAhead = 4;
+    bool bad_page = false;
     auto issue = [&](int i) {
       const int buf = i % NS;
       const int r0 = i * kStageRows, nr = min(kStageRows, seg_len - r0);
+      const int ta = (int)(t0 + r0), tb = ta + nr, P = p.page_size;  // token offsets < 2^31
+      const int lp0 = (int)((uint32_t)ta / (uint32_t)P) + lane, lp_end = (int)((uint32_t)(tb - 1) / (uint32_t)P);
+      int64_t row[kLookAhead];
+#pragma unroll
+      for (int k = 0; k < kLookAhead; ++k) {
+        const int lp = lp0 + 32 * k;
+        row[k] = lp <= lp_end ? cache_row(p, b, kvh, max(ta, lp * P), bad_page) : 0;
+      }
       if (lane == 0) {
         if (i >= NS && !mbar_wait_timed(&sm_empty[buf], (uint32_t)((i / NS) - 1) & 1u, kWaitNs))
           atomicOr(p.err, kErrTimeout);
@@ -195,10 +208,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_ext_kernel(const Deco
       __syncwarp();
       if (i == p.withhold) return;  // test hook: this stage never arrives
       unsigned char* dst = ring + (size_t)buf * kStageBytes;
-      const int64_t ta = t0 + r0, tb = ta + nr, P = p.page_size;
-      for (int64_t lp = ta / P + lane; lp <= (tb - 1) / P; lp += 32) {
-        const int64_t s0 = max(ta, lp * P), s1 = min(tb, (lp + 1) * P);
-        bulk_copy_g2s(dst + (s0 - ta) * kCodeBytes, p.codes + cache_row(p, b, kvh, s0) * kCodeBytes,
+#pragma unroll
+      for (int k = 0; k < kLookAhead; ++k) {
+        const int lp = lp0 + 32 * k;
+        if (lp <= lp_end) {
+          const int s0 = max(ta, lp * P), s1 = min(tb, (lp + 1) * P);
+          bulk_copy_g2s(dst + (size_t)(s0 - ta) * kCodeBytes, p.codes + row[k] * kCodeBytes,
+                        (uint32_t)(s1 - s0) * kCodeBytes, &sm_full[buf]);
+        }
+      }
+      for (int lp = lp0 + 32 * kLookAhead; lp <= lp_end; lp += 32) {  // pages of fewer than 8 tokens
+        const int s0 = max(ta, lp * P), s1 = min(tb, (lp + 1) * P);
+        bulk_copy_g2s(dst + (size_t)(s0 - ta) * kCodeBytes, p.codes + cache_row(p, b, kvh, s0, bad_page) * kCodeBytes,
                       (uint32_t)(s1 - s0) * kCodeBytes, &sm_full[buf]);
       }
     };
@@ -216,6 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_ext_kernel(const Deco
         }
     } else {
       for (int i = 0; i < nst; ++i) issue(i);
+      if (bad_page) atomicOr(p.err, kErrTable);
     }
     __syncwarp();
     cluster_wait();
@@ -584,10 +606,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_ext_kernel(const Deco
       // paged cache: the kept offsets [0, n) become cache rows (one table lookup each)
       auto to_rows = [&](int n) {
         if (!paged) return;
+        bool bad = false;
         for (int i = tid; i < n; i += kWorkers) {
           const uint32_t off = lds32(smem_addr(sm_kept + i)) & kPosMask;
-          sm_kept[i] = (int32_t)cache_row(p, b, kvh, t0 + off);
+          sm_kept[i] = (int32_t)cache_row(p, b, kvh, t0 + off, bad);
         }
+        if (bad) atomicOr(p.err, kErrTable);
         worker_sync();
       };
       // gather of the kept tokens [0, n) of one window into the softmax state
