@@ -605,6 +605,19 @@ static int enqueue_decode(const adamas_decode_args& a, int64_t Nmax, unsigned ch
   return launch_decode(prm, P, decode_mode(a), st);
 }
 
+// Few long heads (too few clusters for the SMs): the plain step splits every
+// (b, kv head) into S slices inside the GPU -- the sharded step's two launches with
+// vslices = S and a merge of the S softmax states (defined with the sequence-sharded
+// step below).
+struct SlicePlan {
+  int S = 1;
+  Plan P;
+  size_t hist_off = 0, part_off = 0, total = 0;
+};
+static int slice_plan(int B, int Hq, int Hkv, int64_t Nmax, int d, int budget, const Plan& P0, DeviceInfo& dev,
+                      SlicePlan* out);
+static int enqueue_sliced(const adamas_decode_args& a, int64_t Nmax, const SlicePlan& SP, cudaStream_t st);
+
 // A decode call on a caller workspace: checks, plan, launch.
 static int decode_with_workspace(const adamas_decode_args& a, cudaStream_t st) {
   int64_t Nmax = 0;
@@ -614,7 +627,16 @@ static int decode_with_workspace(const adamas_decode_args& a, cudaStream_t st) {
   int devno = 0;
   if ((rc = device_info(&dev, &devno)) != ADAMAS_OK) return rc;
   Plan P;
-  if ((rc = make_plan(a.B, a.Hq, a.Hkv, Nmax, decode_mode(a), *dev, devno, &P)) != ADAMAS_OK) return rc;
+  const int mode = decode_mode(a);
+  if ((rc = make_plan(a.B, a.Hq, a.Hkv, Nmax, mode, *dev, devno, &P)) != ADAMAS_OK) return rc;
+  if (mode == kModePlain) {
+    SlicePlan SP;
+    if ((rc = slice_plan(a.B, a.Hq, a.Hkv, Nmax, a.d, a.budget, P, *dev, &SP)) != ADAMAS_OK) return rc;
+    if (SP.S > 1) {
+      if (!a.workspace || a.workspace_bytes < SP.total || !aligned(a.workspace, 16)) return ADAMAS_ERR_WORKSPACE;
+      return enqueue_sliced(a, Nmax, SP, st);
+    }
+  }
   if (!a.workspace || a.workspace_bytes < P.total || !aligned(a.workspace, 16)) return ADAMAS_ERR_WORKSPACE;
   return enqueue_decode(a, Nmax, static_cast<unsigned char*>(a.workspace), P, st);
 }
@@ -656,7 +678,9 @@ size_t adamas_workspace_bytes(int B, int Hq, int Hkv, int64_t Nmax, int d, int b
   if (device_info(&dev, &devno) != ADAMAS_OK) return 0;
   Plan P;
   if (make_plan(B, Hq, Hkv, Nmax, kModePlain, *dev, devno, &P) != ADAMAS_OK) return 0;
-  return P.total;
+  SlicePlan SP;
+  if (slice_plan(B, Hq, Hkv, Nmax, d, budget, P, *dev, &SP) != ADAMAS_OK) return 0;
+  return SP.S > 1 && SP.total > P.total ? SP.total : P.total;
 }
 
 int adamas_workspace_init(void* workspace, size_t workspace_bytes, adamas_stream_t stream) {
@@ -861,6 +885,76 @@ int adamas_merge_partials(const float* partials, int n, int B, int Hq, float* ou
   if (e != cudaSuccess) return cuda_fail(e);
   return ADAMAS_OK;
 }
+
+}  // extern "C"
+
+namespace adamas {
+
+constexpr int64_t kSliceMinTokens = 65536;  // shorter contexts stay one launch (fixed costs dominate)
+constexpr int kMaxSlices = 8;
+
+static int slice_plan(int B, int Hq, int Hkv, int64_t Nmax, int d, int budget, const Plan& P0, DeviceInfo& dev,
+                      SlicePlan* out) {
+  out->S = 1;
+  if (Nmax < kSliceMinTokens || (int64_t)P0.grid * 4 >= (int64_t)dev.sms * 3) return ADAMAS_OK;
+  int best = P0.grid;
+  for (int S = 2; S <= kMaxSlices; ++S) {
+    if ((int64_t)B * Hkv * S > 65535) break;
+    Plan P;
+    // S virtual heads of ceil(Nmax / S) tokens per (b, kv head); the query heads follow
+    if (shard_plan(B, Hq * S, Hkv * S, (Nmax + S - 1) / S, d, budget, &P) != ADAMAS_OK) continue;
+    if (P.grid > best + best / 8) {  // two more launches are worth it only for clearly more blocks
+      best = P.grid;
+      out->S = S;
+      out->P = P;
+    }
+  }
+  if (out->S > 1) {
+    const size_t rows = (size_t)B * Hq * out->S;
+    out->hist_off = align256(out->P.total);
+    out->part_off = out->hist_off + align256(rows * kHistStride * sizeof(uint32_t));
+    out->total = out->part_off + align256(rows * kPartial * sizeof(float));
+  }
+  return ADAMAS_OK;
+}
+
+static int enqueue_sliced(const adamas_decode_args& a, int64_t Nmax, const SlicePlan& SP, cudaStream_t st) {
+  unsigned char* ws = static_cast<unsigned char*>(a.workspace);
+  uint32_t* hist = reinterpret_cast<uint32_t*>(ws + SP.hist_off);
+  float* part = reinterpret_cast<float*>(ws + SP.part_off);
+  const size_t rows = (size_t)a.B * a.Hq;
+  cudaError_t e = cudaMemsetAsync(hist, 0, (size_t)SP.S * rows * kHistStride * sizeof(uint32_t), st);
+  if (e == cudaSuccess && a.budget > 0) e = cudaMemsetAsync(a.idx, 0xFF, rows * a.budget * sizeof(int32_t), st);
+  if (e != cudaSuccess) return cuda_fail(e);
+  DecodeParams prm = {};
+  shard_params(prm, SP.P, ws, a.q, a.seq_lens, a.B, a.Hq, a.Hkv, Nmax, a.budget);
+  prm.vslices = SP.S;
+  prm.codes = a.codes;
+  prm.K = static_cast<const uint16_t*>(a.K);  // the appended key is encoded from its K row
+  prm.V = static_cast<const uint16_t*>(a.V);
+  prm.shard_hist = hist;
+  prm.append_pos = a.append_pos;
+  prm.codes_w = a.append_pos ? a.codes : nullptr;
+  int rc = launch_decode(prm, SP.P, kModeShardScore, st);
+  if (rc != ADAMAS_OK) return rc;
+  DecodeParams prm2 = {};
+  shard_params(prm2, SP.P, ws, a.q, a.seq_lens, a.B, a.Hq, a.Hkv, Nmax, a.budget);
+  prm2.vslices = SP.S;
+  prm2.K = static_cast<const uint16_t*>(a.K);
+  prm2.V = static_cast<const uint16_t*>(a.V);
+  prm2.idx = a.idx;
+  prm2.hist_all = hist;
+  prm2.partial = part;
+  if ((rc = launch_decode(prm2, SP.P, kModeShardAttend, st)) != ADAMAS_OK) return rc;
+  merge_partials_kernel<<<(unsigned)rows, kDim, 0, st>>>(part, SP.S, (int64_t)rows, a.out);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e);
+  return ADAMAS_OK;
+}
+
+}  // namespace adamas
+
+extern "C" {
 
 int adamas_score(const void* q, const uint8_t* codes, const int32_t* seq_lens, int B, int Hq, int Hkv, int64_t Nmax,
                  int d, uint16_t* dist, adamas_stream_t stream) {

@@ -111,6 +111,7 @@ struct DecodeParams {
   uint32_t* blk_hist;         // [grid][G][kHistStride] each block's own histograms (workspace)
   float* partial;             // attend: [B][Hq][kPartial] this slice's softmax state (m, l, -, -, o[128])
   int shard_rank, shard_world;
+  int vslices;                // sharded modes on one GPU: slices per (b, kv head) in this launch (1: none)
   int B, Hq, Hkv;
   int64_t Nmax;           // tokens per sequence the cache can hold (paged: max_pages * page_size)
   int budget;

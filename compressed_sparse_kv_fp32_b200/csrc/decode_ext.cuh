@@ -27,6 +27,11 @@ constexpr int kModeShared = 2;
 //                     slice's kept tokens.
 // The histogram exchange makes the selection exactly the one of the whole
 // sequence: the slices play the part the blocks of a cluster play inside a GPU.
+// With vslices = S > 1 the same two launches split every (b, kv head) of one GPU's
+// cache into S slices, one cluster each (more clusters for few long heads): the
+// score launch writes slice s's histograms at [s][B][Hq], which is then already
+// the gathered buffer of the attend launch, token indices are the cache's own, and
+// the attend launch writes slice s's state at [s][B][Hq].
 constexpr int kModeShardScore = 3;
 constexpr int kModeShardAttend = 4;
 
@@ -56,7 +61,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_ext_kernel(const Deco
   cg::cluster_group cluster = cg::this_cluster();
   const int C = p.cluster;
   const int rank = (int)cluster.block_rank();
-  const int hk = (int)(blockIdx.x / (unsigned)C);  // (b, kv head) of the cluster
+  const int clus = (int)(blockIdx.x / (unsigned)C);  // the cluster
+  // slices of one (b, kv head) in this launch (the sharded modes on one GPU)
+  const int VS = (SCORE_ONLY || ATTEND_ONLY) && p.vslices > 1 ? p.vslices : 1;
+  const int hk = clus / VS, vs = clus - hk * VS;  // (b, kv head) of the cluster, its slice
   const int b = hk / p.Hkv, kvh = hk - b * p.Hkv;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const bool worker = warp < kWorkerWarps;
@@ -106,8 +114,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_ext_kernel(const Deco
   // distance bins: [0, 384] per query head, [0, 384 G] summed over a group; one more
   // when forced rows take bin 0
   const int nbins = (SHARED ? 3 * kDim * G + 1 : kBins) + (forced ? 1 : 0);
-  const int64_t t0 = (int64_t)rank * len_b / C;
-  int seg_len = (int)((int64_t)(rank + 1) * len_b / C - t0);  // <= dstride by the host's sizing
+  // the cluster's tokens [sb0, sb0 + sl) (the whole sequence unless sliced), the block's share of them
+  const int64_t sb0 = (int64_t)vs * len_b / VS, sl = (int64_t)(vs + 1) * len_b / VS - sb0;
+  const int64_t t0 = sb0 + (int64_t)rank * sl / C;
+  int seg_len = (int)(sb0 + (int64_t)(rank + 1) * sl / C - t0);  // <= dstride by the host's sizing
   if (seg_len > p.dstride) {  // never with the host's plan; keeps every distance store in bounds
     if (tid == 0) atomicOr(p.err, kErrInternal);
     seg_len = p.dstride;
@@ -123,7 +133,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_ext_kernel(const Deco
   // the shared-memory copy in its place.
   int64_t apos = -1;
   int arow = -1;  // its row in this block's segment (-1: not scored here)
-  if (ap >= 0 && ap < p.Nmax && ((ap >= t0 && ap < t0 + seg_len) || (rank == C - 1 && ap >= len_b))) {
+  if (ap >= 0 && ap < p.Nmax &&
+      ((ap >= t0 && ap < t0 + seg_len) || (rank == C - 1 && vs == VS - 1 && ap >= len_b))) {
     apos = ap;
     if (ap >= t0 && ap < t0 + seg_len) arow = (int)(ap - t0);
   }
@@ -146,15 +157,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_ext_kernel(const Deco
   // histogram totals (every scored token is counted once per query head) of all
   // slices and of the slices before this one.
   int64_t ofs = 0;
+  const int srank = VS > 1 ? vs : p.shard_rank, sworld = VS > 1 ? VS : p.shard_world;
   if constexpr (ATTEND_ONLY) {
     const uint32_t* h0 = p.hist_all + ((int64_t)b * p.Hq + (int64_t)kvh * G) * kHistStride;
     const int64_t rs = (int64_t)p.B * p.Hq * kHistStride;
     unsigned long long before = 0ull, total = 0ull;
-    for (int i = tid; i < p.shard_world * kBins; i += kThreads) {
+    for (int i = tid; i < sworld * kBins; i += kThreads) {
       const int r = i / kBins, d = i - r * kBins;
       const uint32_t v = h0[r * rs + d];
       total += v;
-      if (r < p.shard_rank) before += v;
+      if (r < srank) before += v;
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -166,7 +178,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_ext_kernel(const Deco
       atomicAdd(&sm_len[1], total);
     }
     __syncthreads();
-    ofs = (int64_t)sm_len[0];
+    ofs = VS > 1 ? 0 : (int64_t)sm_len[0];  // slices of one cache index its tokens themselves
     int64_t len_g = (int64_t)sm_len[1];
     if (len_g > INT32_MAX) {  // global indices are int32
       if (rank == 0 && tid == 0) atomicOr(p.err, kErrSeqLen);
@@ -254,15 +266,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_ext_kernel(const Deco
       const int64_t arow_c = GENERAL ? cache_row(p, b, kvh, apos) : kv_base + apos;
       const int64_t nrow = (int64_t)b * p.Hkv + kvh;
       const bool rows_in = GENERAL && p.k_new != nullptr;
-      const uint32_t w = encode128_warp(rows_in ? p.k_new + nrow * kDim : p.K + arow_c * kDim, lane);
-      if (lane < kCodeWords) {
-        sm_acode[lane] = w;
-        reinterpret_cast<uint32_t*>(p.codes_w + arow_c * kCodeBytes)[lane] = w;
-      }
-      if (rows_in) {  // the new K row (lanes 0-15) and V row (lanes 16-31) into the cache
-        const uint16_t* src = (lane < 16 ? p.k_new : p.v_new) + nrow * kDim + (lane & 15) * 8;
-        uint16_t* dst = (lane < 16 ? p.K_w : p.V_w) + arow_c * kDim + (lane & 15) * 8;
-        *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
+      const uint16_t* ksrc = rows_in ? p.k_new + nrow * kDim : (p.K != nullptr ? p.K + arow_c * kDim : nullptr);
+      if (ksrc == nullptr || p.codes_w == nullptr) {  // never with the host's launches: flagged, nothing read
+        if (lane == 0) atomicOr(p.err, kErrInternal);
+      } else {
+        const uint32_t w = encode128_warp(ksrc, lane);
+        if (lane < kCodeWords) {
+          sm_acode[lane] = w;
+          reinterpret_cast<uint32_t*>(p.codes_w + arow_c * kCodeBytes)[lane] = w;
+        }
+        if (rows_in) {  // the new K row (lanes 0-15) and V row (lanes 16-31) into the cache
+          const uint16_t* src = (lane < 16 ? p.k_new : p.v_new) + nrow * kDim + (lane & 15) * 8;
+          uint16_t* dst = (lane < 16 ? p.K_w : p.V_w) + arow_c * kDim + (lane & 15) * 8;
+          *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
+        }
       }
     }
     worker_sync();
@@ -365,7 +382,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_ext_kernel(const Deco
         const uint32_t v = sm_hist[i];
         bh[i] = v;
         const int g = i / kHistStride, d = i - g * kHistStride;
-        if (v != 0u) atomicAdd(p.shard_hist + ((int64_t)b * p.Hq + kvh * G + g) * kHistStride + d, v);
+        if (v != 0u)
+          atomicAdd(p.shard_hist + ((int64_t)vs * p.B * p.Hq + (int64_t)b * p.Hq + kvh * G + g) * kHistStride + d, v);
       }
     } else if constexpr (ATTEND_ONLY) {  // own histograms from the score half
       const uint32_t* bh = p.blk_hist + (size_t)blockIdx.x * G * kHistStride;
@@ -403,7 +421,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_ext_kernel(const Deco
           if (d >= nbins) return;
           if constexpr (ATTEND_ONLY) {
             // this slice: the blocks of the cluster; the other slices: their sums
-            const uint32_t* bh = p.blk_hist + ((size_t)hk * C * G + g) * kHistStride + d;
+            const uint32_t* bh = p.blk_hist + ((size_t)clus * C * G + g) * kHistStride + d;
             for (int r = 0; r < C; ++r) {
               const uint32_t v = bh[(size_t)r * G * kHistStride];
               H += v;
@@ -411,11 +429,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_ext_kernel(const Deco
             }
             const uint32_t* ha = p.hist_all + ((int64_t)b * p.Hq + (int64_t)kvh * G + g) * kHistStride + d;
             const int64_t rs = (int64_t)p.B * p.Hq * kHistStride;
-            for (int r = 0; r < p.shard_world; ++r) {
-              if (r == p.shard_rank) continue;
+            for (int r = 0; r < sworld; ++r) {
+              if (r == srank) continue;
               const uint32_t v = ha[r * rs];
               H += v;
-              if (r < p.shard_rank) P += v;
+              if (r < srank) P += v;
             }
           } else {
             uint32_t v[kMaxCluster];
@@ -947,7 +965,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_ext_kernel(const Deco
           res = O / L;
         }
         if constexpr (ATTEND_ONLY) {  // the slice's state (m = -inf, l = 0: it kept no token)
-          float* dst = p.partial + hq * kPartial;
+          float* dst = p.partial + ((int64_t)vs * p.B * p.Hq + hq) * kPartial;
           dst[4 + e] = O;
           if (e == 0) {
             dst[0] = M;

@@ -187,7 +187,10 @@ def test_append_rows_written_by_the_launch(B, Hq, Hkv, N, lens, apos, budget):
     assert ws.device_error() == 0
     assert torch.equal(K, K2) and torch.equal(V, V2) and torch.equal(codes, c2)
     assert torch.equal(idx, ref_idx)
-    assert torch.equal(out.view(torch.int32), ref_out.view(torch.int32))
+    # the same kept rows; the reference may run the sliced step (long context, one kv
+    # head), whose merge of slice states sums in another fp32 order: the outputs agree
+    # within the float tolerance of every parity test
+    assert_close_out(out.cpu().numpy(), ref_out.cpu().numpy())
 
 
 # ---------------------------------------------------------------- every option at once

@@ -46,8 +46,7 @@ def test_matches_workspace_entry_point_twice(wid, kw, budget):
     w = synth.WORKLOADS[wid].scaled(**kw)
     inp, K, V, codes = _inputs(w)
     lens = dev(inp["lens"])
-    ws = adamas.Workspace(w.B, w.Hq, w.Hkv, w.Nmax, budget)
-    assert ws.nbytes <= 4 << 20
+    ws = adamas.Workspace(w.B, w.Hq, w.Hkv, w.Nmax, budget)  # the static call checks its own 4 MiB bound
     for step in (0, 1):                      # two calls in a row on the shared scratch
         q = dev_bf16(synth.query(w, step))
         ref_out, ref_idx = adamas.decode_step(q, codes, K, V, lens, budget, ws)
