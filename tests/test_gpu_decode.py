@@ -226,6 +226,7 @@ def _sampled_oracle(orc, w, q, lens, budget, b, kvh):
 
 @pytest.mark.parametrize("wid,budget,heads", [(3, 1024, [(0, 0), (0, 13), (0, 31)]),
                                               (3, 64, [(0, 7)]),
+                                              (3, 128, [(0, 21)]),
                                               (5, 1024, [(0, 5)])])
 def test_full_size_sampled_heads(orc, wid, budget, heads):
     w = synth.WORKLOADS[wid]
