@@ -88,9 +88,13 @@ const char *adamas_last_error_string(void);
  * current CUDA device (0 when the sizes are unsupported).  The workspace holds
  * the device error word and, only when a block's token distances do not fit in
  * shared memory (very long contexts), a spill area for them; histograms and
- * partial softmax states stay on chip.  It must be zero-filled once before its first use
- * (adamas_workspace_init); every step leaves it ready for the next one.  One
- * workspace must not be used by two steps that may run concurrently.
+ * partial softmax states stay on chip.  For long contexts over few kv heads
+ * (fewer clusters than fill 3/4 of the SMs, at least 65,536 tokens) the step
+ * splits every (b, kv head) into slices inside the GPU, and the workspace also
+ * carries the slices' histograms and softmax states.  It must be zero-filled once
+ * before its first use (adamas_workspace_init); every step leaves it ready for the
+ * next one.  One workspace must not be used by two steps that may run
+ * concurrently.
  */
 size_t adamas_workspace_bytes(int B, int Hq, int Hkv, int64_t Nmax, int d, int budget);
 
