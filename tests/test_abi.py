@@ -106,3 +106,26 @@ def test_decode_ex_rejects_bad_options_before_any_launch(lib):
     assert call(block_table=fake, page_size=0, max_pages=4, n_pages=8) == -1
     assert call(block_table=fake + 2, page_size=16, max_pages=4, n_pages=8) == -1   # misaligned table
     assert lib.adamas_decode_step_ex(None, None) == -1
+
+
+def test_sharded_and_static_calls_reject_bad_arguments_before_any_launch(lib):
+    fake = ctypes.c_void_p(1 << 20)                  # never dereferenced: the checks come first
+    # adamas_shard_score: a null histogram buffer, a misaligned q
+    assert lib.adamas_shard_score(fake, fake, fake, 1, 4, 1, 4096, 128, 64, None, fake, 1 << 20, None) == -1
+    assert lib.adamas_shard_score(ctypes.c_void_p((1 << 20) + 2), fake, fake, 1, 4, 1, 4096, 128, 64, fake, fake,
+                                  1 << 20, None) == -1
+    assert lib.adamas_shard_score(fake, fake, fake, 1, 4, 1, 4096, 64, 64, fake, fake, 1 << 20, None) == -2  # d != 128
+    # adamas_shard_attend: world < 1, rank outside [0, world), a null state buffer
+    def attend(world, rank, partial=fake):
+        return lib.adamas_shard_attend(fake, fake, fake, fake, 1, 4, 1, 4096, 128, 64, fake, world, rank, partial,
+                                       fake, fake, 1 << 20, None)
+    assert attend(0, 0) == -1
+    assert attend(2, 2) == -1
+    assert attend(2, -1) == -1
+    assert attend(2, 1, partial=None) == -1
+    # adamas_merge_partials: no state, a null output, nothing to merge
+    assert lib.adamas_merge_partials(fake, 0, 1, 4, fake, None) == -1
+    assert lib.adamas_merge_partials(fake, 2, 1, 4, None, None) == -1
+    assert lib.adamas_merge_partials(fake, 2, 0, 4, fake, None) == 0
+    # adamas_static_device_error: a null word pointer
+    assert lib.adamas_static_device_error(None, None) == -1
